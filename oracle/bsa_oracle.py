@@ -1,0 +1,341 @@
+"""CPU oracle for training-free block-sparse 3D attention — TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py`` may import this module. The CUDA library never calls it and shares no code
+with it; when the CUDA extension is missing the product path fails instead of falling back
+here.
+
+Plain numpy, float64 arithmetic on the bf16 inputs (widened exactly). Every step is written
+the slow, obvious way, in the order the pages describe the method:
+
+1. ``block_layout``    — tile-major order of the 3D token grid, cut into query/key blocks
+2. ``pool_blocks``     — per-block mean of Q or K over the block's real tokens
+3. ``score_meanpool``  — softmax over key blocks of the pooled-query . pooled-key logits
+   ``score_park``      — each query softmaxed over key blocks, then averaged in its block
+4. ``select_topp``     — per-row top-p kept-block list (score descending, index ascending)
+5. ``drift``           — per-head relative Q/K change since the cached reference
+6. ``sparse_attention``— exact softmax attention restricted to the kept key blocks
+7. ``reuse_run``       — the drift-gated mask-reuse loop across denoising steps
+
+Sources (page title, then the part of the page):
+* PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers —
+  Abstract: retrieval by averaged query/key block representations (the mean-pooled
+  estimate), PARK's per-query normalisation over key blocks averaged within the query
+  block, and attention computed only within the retrieved blocks.
+* HASTE: Training-Free Video Diffusion Acceleration via Head-Wise Adaptive Sparse
+  Attention — abstract: online top-p block selection, per-head thresholds, mask
+  prediction skipped on small query-key drift.
+* HEART: Exploiting Head Heterogeneity in Sparse Attention for Video Diffusion —
+  abstract: Temporal Mask Reuse refreshes a head's cached mask only when its query-key
+  drift exceeds a prescribed threshold.
+* RAPID: Reusing Attention Sparsity with Inter-step Adaptation for Efficient Video
+  Diffusion — English abstract: 3D attention, block importance estimated and the sparse
+  mask cached for reuse across steps.
+
+Where the pages are silent the plainest reading is taken; each one is named at the point
+of use (block shape/order, logit scale, top-p boundary, tie order, text blocks, drift
+norm).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bit patterns (uint16) to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def default_tile(block: int):
+    """Tile (t, h, w) that holds exactly one block: 1x8x8 for 64 tokens, 2x8x8 for 128.
+
+    Reading: the pages speak of query and key blocks of a 3D token grid (PARK abstract;
+    RAPID abstract, "3D attention") without a shape; a cube-like 3D tile is the plainest
+    choice.
+    """
+    if block == 64:
+        return (1, 8, 8)
+    if block == 128:
+        return (2, 8, 8)
+    raise ValueError("block must be 64 or 128")
+
+
+# ----------------------------------------------------------------------- 1. block layout
+
+@dataclasses.dataclass
+class Layout:
+    perm: np.ndarray       # int64 [nb*B]: raster token index per slot, -1 for padding
+    B: int
+    nb: int                # total blocks
+    nb_video: int          # video blocks (the last one may be partial)
+    nb_text: int           # text blocks (after the padded video part)
+    counts: np.ndarray     # int64 [nb]: real tokens per block
+
+    @property
+    def npad(self) -> int:
+        return self.nb * self.B
+
+    def rows(self, i: int) -> np.ndarray:
+        """Raster token indices of the real tokens of block i, in block order."""
+        s = self.perm[i * self.B:(i + 1) * self.B]
+        return s[s >= 0]
+
+    def is_text_block(self, i: int) -> bool:
+        return i >= self.nb_video
+
+
+def block_layout(T: int, H: int, W: int, text_tokens: int, block: int, tile=None) -> Layout:
+    """Tile-major order of the video grid, cut into blocks of `block` tokens.
+
+    Reading: tiles of shape (tt, th, tw) are visited in raster order of their tile
+    coordinates; the tokens of a tile are taken in raster order (t, y, x; x fastest), edge
+    tiles keep only the tokens inside the grid. The concatenated order is cut into blocks of
+    B consecutive tokens, so only the last video block can be partial; it is padded. Text
+    tokens (raster indices after the video tokens) follow as their own blocks, the last one
+    padded.
+    """
+    tt, th, tw = tile if tile is not None else default_tile(block)
+    order = []
+    for a in range(0, T, tt):
+        for b in range(0, H, th):
+            for c in range(0, W, tw):
+                for t in range(a, min(a + tt, T)):
+                    for y in range(b, min(b + th, H)):
+                        for x in range(c, min(c + tw, W)):
+                            order.append((t * H + y) * W + x)
+    nv = T * H * W
+    nbv = -(-nv // block) if nv > 0 else 0
+    nbt = -(-text_tokens // block) if text_tokens > 0 else 0
+    nb = nbv + nbt
+    perm = np.full(nb * block, -1, dtype=np.int64)
+    perm[:nv] = np.asarray(order, dtype=np.int64)
+    perm[nbv * block:nbv * block + text_tokens] = nv + np.arange(text_tokens, dtype=np.int64)
+    counts = np.array([(perm[i * block:(i + 1) * block] >= 0).sum() for i in range(nb)],
+                      dtype=np.int64)
+    return Layout(perm, block, nb, nbv, nbt, counts)
+
+
+# --------------------------------------------------------------------------- 2. pooling
+
+def pool_blocks(X: np.ndarray, layout: Layout) -> np.ndarray:
+    """Mean of X's rows over each block's real tokens (padding excluded; divide by the real
+    count). X is float64 [N, d] in raster order; returns [nb, d].
+    (PARK abstract: "averaged representations of query and key blocks".)"""
+    out = np.zeros((layout.nb, X.shape[1]), dtype=np.float64)
+    for i in range(layout.nb):
+        r = layout.rows(i)
+        out[i] = X[r].sum(axis=0) / len(r)
+    return out
+
+
+# --------------------------------------------------------------------------- 3. scoring
+
+def _softmax_rows(L: np.ndarray) -> np.ndarray:
+    """Row softmax, two passes: subtract the row max, exponentiate, divide by the sum."""
+    m = L.max(axis=1, keepdims=True)
+    e = np.exp(L - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def score_meanpool(Qh: np.ndarray, Kh: np.ndarray, layout: Layout) -> np.ndarray:
+    """S[i, j] = softmax over j of (qbar_i . kbar_j) / sqrt(d), all key blocks j.
+
+    The mean-pooled retrieval estimate the PARK abstract describes (query and key blocks
+    represented by their averages). Reading: the logit scale is 1/sqrt(d), the same as the
+    attention it predicts; no size correction for partial blocks.
+    """
+    d = Qh.shape[1]
+    qbar = pool_blocks(Qh, layout)
+    kbar = pool_blocks(Kh, layout)
+    return _softmax_rows(qbar @ kbar.T / math.sqrt(d))
+
+
+def score_park(Qh: np.ndarray, Kh: np.ndarray, layout: Layout) -> np.ndarray:
+    """P[i, j] = mean over real queries q of block i of softmax_j(q . kbar_j / sqrt(d)).
+
+    PARK abstract: every original query is kept, its attention over key blocks is
+    normalised on its own, and those distributions are averaged within the query block.
+    Reading: key blocks are represented by their mean key (the page's query-aware key
+    clustering has no formula there and is not part of this scorer).
+    """
+    d = Qh.shape[1]
+    kbar = pool_blocks(Kh, layout)
+    P = np.zeros((layout.nb, layout.nb), dtype=np.float64)
+    for i in range(layout.nb):
+        q = Qh[layout.rows(i)]
+        P[i] = _softmax_rows(q @ kbar.T / math.sqrt(d)).mean(axis=0)
+    return P
+
+
+# ------------------------------------------------------------------------ 4. top-p select
+
+def sort_row(scores_row_f32: np.ndarray) -> np.ndarray:
+    """Block indices ordered by score descending, then index ascending."""
+    s = np.asarray(scores_row_f32, dtype=np.float32).astype(np.float64)
+    j = np.arange(len(s))
+    return np.lexsort((j, -s))
+
+
+def select_row(scores_row_f32: np.ndarray, p: float, forced=()):
+    """Top-p kept list for one (head, query-block) row.
+
+    HASTE abstract (online top-p block selection, per-head thresholds). Readings:
+    * blocks are ordered by score descending, ties by index ascending;
+    * the kept prefix is the shortest one whose cumulative score reaches p (>= p), so at
+      least one block is kept; p >= 1 keeps every block (float32 sums may stop short of 1);
+    * the cumulative sum is taken in float32, sequentially in sorted order (float32 is the
+      precision of the stored scores and of the kernel that makes the same decision);
+    * forced blocks (text key blocks) are added to the kept set, and the union keeps the
+      same order.
+    Returns (kept list, sorted order, float32 cumulative masses in sorted order).
+    """
+    s32 = np.asarray(scores_row_f32, dtype=np.float32)
+    order = sort_row(s32)
+    cum = np.cumsum(s32[order], dtype=np.float32)
+    n = len(order)
+    if p >= 1.0:
+        m = n
+    else:
+        hit = np.nonzero(cum >= np.float32(p))[0]
+        m = int(hit[0]) + 1 if len(hit) else n
+    keep = np.zeros(n, dtype=bool)
+    keep[order[:m]] = True
+    keep[np.asarray(list(forced), dtype=np.int64)] = True
+    kept = [int(j) for j in order[keep[order]]]
+    return kept, order, cum
+
+
+def select_topp(scores_f32: np.ndarray, p: float, layout: Layout):
+    """Kept-block lists for every query block of one head.
+
+    Text query blocks keep every block; video query blocks keep their top-p set plus all
+    text key blocks (reading of "text tokens always kept as dense key/query blocks").
+    Returns idx int32 [nb, nb] (entries past cnt are -1) and cnt int32 [nb].
+    """
+    nb = layout.nb
+    idx = np.full((nb, nb), -1, dtype=np.int32)
+    cnt = np.zeros(nb, dtype=np.int32)
+    text = list(range(layout.nb_video, nb))
+    for i in range(nb):
+        if layout.is_text_block(i):
+            kept, _, _ = select_row(scores_f32[i], 1.0)
+        else:
+            kept, _, _ = select_row(scores_f32[i], p, forced=text)
+        idx[i, :len(kept)] = kept
+        cnt[i] = len(kept)
+    return idx, cnt
+
+
+# ------------------------------------------------------------------------------ 5. drift
+
+def relative_change(X: np.ndarray, Xref: np.ndarray) -> float:
+    """||X - Xref||_F / ||Xref||_F (0 when both are zero, +inf when only Xref is)."""
+    num = math.sqrt(float(((X - Xref) ** 2).sum()))
+    den = math.sqrt(float((Xref ** 2).sum()))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else math.inf
+    return num / den
+
+
+def drift(Qh, Kh, Qref_h, Kref_h) -> float:
+    """Per-head query-key drift since the head's last refresh (HEART abstract, Temporal
+    Mask Reuse). Reading: the larger of the relative Frobenius changes of Q and K over the
+    head's real tokens."""
+    return max(relative_change(Qh, Qref_h), relative_change(Kh, Kref_h))
+
+
+def refresh_decision(delta: float, tau: float, have_cache: bool) -> bool:
+    """Refresh when there is no cached mask yet or the drift is strictly above tau."""
+    return (not have_cache) or (delta > tau)
+
+
+# -------------------------------------------------------------------------- 6. attention
+
+def sparse_attention_head(Qh, Kh, Vh, idx, cnt, layout: Layout, qblocks=None) -> np.ndarray:
+    """O_t = sum over real keys u of the kept blocks of softmax_u(Q_t . K_u / sqrt(d)) V_u.
+
+    The exact definition of attention restricted to the retrieved blocks (PARK abstract:
+    attention computed only within the retrieved blocks). Logits over the kept real keys
+    are materialised, softmaxed in two passes (max, then sum) and applied to V. Rows of
+    query blocks not listed in `qblocks` are left as NaN. Returns float64 [N, d] in raster
+    order.
+    """
+    N, d = Qh.shape
+    O = np.full((N, Vh.shape[1]), np.nan, dtype=np.float64)
+    scale = 1.0 / math.sqrt(d)
+    for i in (range(layout.nb) if qblocks is None else qblocks):
+        rows = layout.rows(i)
+        keys = np.concatenate([layout.rows(int(j)) for j in idx[i, :cnt[i]]])
+        L = (Qh[rows] @ Kh[keys].T) * scale
+        m = L.max(axis=1, keepdims=True)
+        e = np.exp(L - m)
+        O[rows] = (e @ Vh[keys]) / e.sum(axis=1, keepdims=True)
+    return O
+
+
+# ----------------------------------------------------------------------- whole pipeline
+
+def score_head(Qh, Kh, layout, mode: str) -> np.ndarray:
+    if mode == "meanpool":
+        return score_meanpool(Qh, Kh, layout)
+    if mode == "park":
+        return score_park(Qh, Kh, layout)
+    raise ValueError(mode)
+
+
+def pipeline_head(Qb, Kb, Vb, layout, p, mode="meanpool", qblocks=None):
+    """Score -> select -> attend for one head (bf16 bit inputs [N, d]).
+    Returns (scores float32 [nb, nb], idx, cnt, O float64 [N, d])."""
+    Qh, Kh, Vh = bf16_to_f64(Qb), bf16_to_f64(Kb), bf16_to_f64(Vb)
+    S = score_head(Qh, Kh, layout, mode).astype(np.float32)
+    idx, cnt = select_topp(S, p, layout)
+    O = sparse_attention_head(Qh, Kh, Vh, idx, cnt, layout, qblocks)
+    return S, idx, cnt, O
+
+
+# --------------------------------------------------------------------- 7. mask-reuse run
+
+def reuse_run(steps_qk, V, layout, p, tau, mode="meanpool", attend=True):
+    """Drift-gated mask reuse across denoising steps (HEART abstract, Temporal Mask Reuse;
+    HASTE abstract; RAPID abstract: masks cached and reused across steps).
+
+    `steps_qk` yields (Q, K) bf16 bits [heads, N, d] per step; V is fixed. At each step a
+    head whose drift since its last refresh exceeds tau (or that has no cache yet) re-scores,
+    re-selects and snapshots its Q, K as the new reference; the other heads reuse their
+    cached kept lists. Returns a dict with per-step drift, refresh flags, the final masks
+    and (if `attend`) the per-step outputs.
+    """
+    heads = V.shape[0]
+    Vf = [bf16_to_f64(V[h]) for h in range(heads)]
+    ref = [None] * heads
+    masks = [None] * heads
+    out = {"drift": [], "refresh": [], "O": []}
+    for Q, K in steps_qk:
+        deltas, flags, Os = [], [], []
+        for h in range(heads):
+            Qh, Kh = bf16_to_f64(Q[h]), bf16_to_f64(K[h])
+            if ref[h] is None:
+                delta = math.inf
+            else:
+                delta = drift(Qh, Kh, ref[h][0], ref[h][1])
+            fresh = refresh_decision(delta, tau, ref[h] is not None)
+            if fresh:
+                S = score_head(Qh, Kh, layout, mode).astype(np.float32)
+                masks[h] = select_topp(S, p[h], layout)
+                ref[h] = (Qh, Kh)
+            deltas.append(delta)
+            flags.append(fresh)
+            if attend:
+                Os.append(sparse_attention_head(Qh, Kh, Vf[h], masks[h][0], masks[h][1], layout))
+        out["drift"].append(deltas)
+        out["refresh"].append(flags)
+        if attend:
+            out["O"].append(np.stack(Os))
+    out["masks"] = masks
+    return out
