@@ -1,0 +1,384 @@
+"""Benchmark of the block-sparse 3D attention hot path on B200.
+
+One step = one pass of the whole path over one layer of synthetic input resident in HBM:
+    drift check (forced refresh: every head re-scores) -> block scores -> top-p select
+    -> block-sparse attention
+on the Wan2.1-1.3B-shaped 480p layer (12 heads, d=128, 21x30x52 grid, 128-token blocks,
+p=0.9) unless --workload says otherwise. Three input sets rotate between steps (900 MB >
+126 MB L2), so no step finds its inputs in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--mode meanpool|park]
+
+Prints one JSON line. Multi-GPU (torchrun): each rank runs its own layer (replicas of the
+same shape, no collective on the data path); value = max-over-ranks step time divided by
+the calls all ranks made (ms per call, whole job).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per sparse-attn call & % bf16 tensor peak (score+select+attend), 1 B200"
+UNIT = "ms"
+TAU = 0.05
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_query_b200 import bsa, inputs
+    from block_sparse_attention_query_b200.layer import SparseAttentionLayer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = inputs.workload(args.workload)
+    mode = bsa.BSA_SCORE_PARK if args.mode == "park" else bsa.BSA_SCORE_MEANPOOL
+    n_sets = 3
+    sets = []
+    for s in range(n_sets):
+        Qb, Kb, Vb = inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=s + 17 * rank)
+        sets.append(tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (Qb, Kb, Vb)))
+    layer = SparseAttentionLayer(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, p=list(w.p),
+                                 tau=TAU, score_mode=mode, device=dev)
+    O = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    prob, plan = layer.prob, layer.plan
+
+    def step(k, ev=None):
+        Q, K, V = sets[k % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        bsa.bsa_drift_check(prob, Q, K, layer.Q_ref, layer.K_ref, TAU, 1, layer.drift, layer.refresh, layer.ws_drift)
+        if ev is not None:
+            ev[1].record(stream)
+        bsa.bsa_score_blocks(prob, Q, K, layer.refresh, layer.scores, layer.ws_score)
+        if ev is not None:
+            ev[2].record(stream)
+        bsa.bsa_select_topp(prob, layer.scores, layer.p, layer.refresh, layer.idx, layer.cnt)
+        if ev is not None:
+            ev[3].record(stream)
+        bsa.bsa_sparse_attention(prob, Q, K, V, layer.idx, layer.cnt, O, layer.ws_attn)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    st = bsa.bsa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(k, evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    stage_ms = np.zeros(4)
+    for e in evs:
+        for s in range(4):
+            stage_ms[s] += e[s].elapsed_time(e[s + 1])
+    stage_ms /= args.steps
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    st = bsa.bsa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    # work accounting from the masks the last step produced
+    cnt = layer.cnt.cpu().numpy().astype(np.int64)
+    kept_pairs = int(cnt.sum())
+    B, d, N, H = w.block, w.d, w.tokens, w.heads
+    att_flops = kept_pairs * 4.0 * B * B * d
+    dense_flops = 4.0 * N * N * d * H
+    elem = 2
+    bytes_qkvo = 4.0 * H * N * d * elem
+    bytes_drift = 6.0 * H * N * d * elem              # read Q,K,Qref,Kref; write Qref,Kref
+    bytes_score = 2.0 * H * N * d * elem              # read Q,K once (pooling)
+    hbm, bf16_peak, bf16_sus, peak_src = _peaks()
+
+    stages = {}
+    names = ["drift_check", "score_blocks", "select_topp", "sparse_attention"]
+    for s, n in enumerate(names):
+        stages[n] = {"ms": round(float(stage_ms[s]), 5), "share": round(float(stage_ms[s] / stage_ms.sum()), 4)}
+    att_s = stage_ms[3] * 1e-3
+    stages["sparse_attention"].update({
+        "tflops_actual": round(att_flops / att_s / 1e12, 2),
+        "tflops_dense_equiv": round(dense_flops / att_s / 1e12, 2),
+        "frac_bf16_peak": round(att_flops / att_s / 1e12 / bf16_peak, 4),
+        "hbm_gbs_compulsory": round(bytes_qkvo / att_s / 1e9, 1),
+        "frac_hbm": round(bytes_qkvo / att_s / 1e9 / hbm, 4)})
+    stages["drift_check"].update({"gbs": round(bytes_drift / (stage_ms[0] * 1e-3) / 1e9, 1),
+                                  "frac_hbm": round(bytes_drift / (stage_ms[0] * 1e-3) / 1e9 / hbm, 4)})
+    stages["score_blocks"].update({"gbs": round(bytes_score / (stage_ms[1] * 1e-3) / 1e9, 1),
+                                   "frac_hbm": round(bytes_score / (stage_ms[1] * 1e-3) / 1e9 / hbm, 4)})
+
+    # dominant kernel roofline
+    dom = names[int(np.argmax(stage_ms))]
+    if dom == "sparse_attention":
+        t_tensor = att_flops / (bf16_peak * 1e12)
+        t_hbm = bytes_qkvo / (hbm * 1e9)
+        if t_tensor >= t_hbm:
+            ach = att_flops / att_s / 1e12
+            roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                    "frac": round(ach / bf16_peak, 4)}
+        else:
+            ach = bytes_qkvo / att_s / 1e9
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(ach / hbm, 4)}
+    else:
+        b = bytes_drift if dom == "drift_check" else bytes_score
+        ach = b / (stage_ms[names.index(dom)] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4)}
+    roof.update({"kernel": dom, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
+                 "traffic": args.traffic})
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in sets[0])
+        for hx, dx in zip((hQ, hK, hV), sets[0]):
+            hx.copy_(dx)
+        hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        Qd, Kd, Vd = (torch.empty_like(x) for x in sets[0])
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            Qd.copy_(hQ, non_blocking=True); Kd.copy_(hK, non_blocking=True); Vd.copy_(hV, non_blocking=True)
+            layer.step(Qd, Kd, Vd, O, force_refresh=True)
+            hO.copy_(O, non_blocking=True)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            Qd.copy_(hQ, non_blocking=True); Kd.copy_(hK, non_blocking=True); Vd.copy_(hV, non_blocking=True)
+            layer.step(Qd, Kd, Vd, O, force_refresh=True)
+            hO.copy_(O, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / e2e_steps
+        if ws > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(e2e_ms / ws, 4), "unit": UNIT,
+               "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
+
+    launches_per_step = 2 + 2 + 1 + 1 + (1 if plan.nb_text > 0 else 0)
+    value = ms_step / ws
+    line = {
+        "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded RFF-structured Q/K, Gaussian V; no model weights)",
+        "config": {"workload": w.name, "heads": H, "d": d, "grid": [w.T, w.H, w.W],
+                   "text_tokens": w.text_tokens, "tokens": N, "block": B, "blocks": plan.nb,
+                   "top_p": sorted(set(float(x) for x in w.p)), "scorer": args.mode,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "3 rotating input sets (%.0f MB each) > 126 MB L2; no flush" % (3 * H * N * d * elem / 1e6),
+                   "step": "drift_check(force) + score_blocks + select_topp + sparse_attention"},
+        "pct_bf16_peak_call": round(100.0 * att_flops / (ms_step * 1e-3) / 1e12 / bf16_peak, 3),
+        "kept_blocks_per_row": round(kept_pairs / (H * plan.nb), 3),
+        "kept_density": round(kept_pairs / (H * plan.nb * plan.nb), 5),
+        "tflops_actual_call": round(att_flops / (ms_step * 1e-3) / 1e12, 2),
+        "tflops_dense_equiv_call": round(dense_flops / (ms_step * 1e-3) / 1e12, 2),
+        "stages": stages, "roofline": roof, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+    }
+    return line, (w, sets if rank == 0 else None)
+
+
+# ------------------------------------------------------------------------- oracle
+
+def oracle_call_ms(w, Qb, Kb, Vb, mode, heads_sample):
+    """Time the oracle's drift + score + select + attention on a sample of heads; returns
+    (ms per call extrapolated to all heads, seconds spent, heads used)."""
+    from oracle import bsa_oracle as O
+    L = O.block_layout(w.T, w.H, w.W, w.text_tokens, w.block)
+    t = time.perf_counter()
+    for h in heads_sample:
+        Qh, Kh, Vh = O.bf16_to_f64(Qb[h]), O.bf16_to_f64(Kb[h]), O.bf16_to_f64(Vb[h])
+        O.drift(Qh, Kh, Qh, Kh)
+        S = O.score_head(Qh, Kh, L, mode).astype(np.float32)
+        idx, cnt = O.select_topp(S, w.p[h], L)
+        O.sparse_attention_head(Qh, Kh, Vh, idx, cnt, L)
+    dt = time.perf_counter() - t
+    return dt / len(heads_sample) * w.heads * 1e3, dt, len(heads_sample)
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args):
+    from block_sparse_attention_query_b200 import inputs
+    w = inputs.workload(args.workload)
+    Qb, Kb, Vb = inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=0)
+    mode = "park" if args.mode == "park" else "meanpool"
+    per_step = []
+    for k in range(args.warmup + args.steps):
+        h = k % w.heads
+        ms, _, _ = oracle_call_ms(w, Qb, Kb, Vb, mode, [h])
+        if k >= args.warmup:
+            per_step.append(ms)
+    v = float(np.mean(per_step))
+    cores = cpu_threads()
+    sample = f"1 of {w.heads} heads per step (full drift+score+select+attention of that head), extrapolated x{w.heads}"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "scorer": mode, "parallelism": "single process (host cores)"},
+        "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan13b_480p")
+    ap.add_argument("--mode", default="meanpool", choices=["meanpool", "park"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=3, help="heads in the bounded oracle sample")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture (None if stale)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank, local = _dist()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from block_sparse_attention_query_b200 import build
+    if rank == 0 or ws == 1:
+        build.build()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    line, (w, sets) = run_ours(args, ws, rank, local)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            import torch
+            Qb, Kb, Vb = (x.view(torch.int16).cpu().numpy().view(np.uint16) for x in sets[0])
+            heads = list(range(min(args.cpu_heads, w.heads)))
+            ms, secs, nh = oracle_call_ms(w, Qb, Kb, Vb, "park" if args.mode == "park" else "meanpool", heads)
+            line["cpu_baseline"] = {"value": round(ms, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                    "sample": f"{nh} of {w.heads} heads, full drift+score+select+attention, "
+                                              f"{secs:.1f} s of CPU work, extrapolated to all heads"}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,296 @@
+// libbsa host side: argument validation, planning and kernel launches behind the C ABI of
+// include/bsa.h. Single translation unit so that the device error word is shared by every
+// kernel of the library.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "bsa_common.cuh"
+#include "score.cuh"
+#include "park.cuh"
+#include "select.cuh"
+#include "drift.cuh"
+#include "attention.cuh"
+
+using namespace bsa;
+
+namespace {
+
+constexpr int kMaxBlocks = 2048;   // top-p sorts at most 2048 keys per row in shared memory
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int resolve_tile(const bsa_problem& pr, int* tt, int* th, int* tw) {
+    if (pr.tile_t == 0 && pr.tile_h == 0 && pr.tile_w == 0) {
+        *tt = pr.block == 64 ? 1 : 2;
+        *th = 8;
+        *tw = 8;
+        return BSA_OK;
+    }
+    if (pr.tile_t < 1 || pr.tile_h < 1 || pr.tile_w < 1) return BSA_ERR_ARG;
+    if ((long long)pr.tile_t * pr.tile_h * pr.tile_w != pr.block) return BSA_ERR_ARG;
+    *tt = pr.tile_t;
+    *th = pr.tile_h;
+    *tw = pr.tile_w;
+    return BSA_OK;
+}
+
+// Validates the problem and fills the device geometry.
+int make_geom(const bsa_problem* prob, Geom* g) {
+    if (prob == nullptr) return BSA_ERR_ARG;
+    const bsa_problem& pr = *prob;
+    if (pr.d != 64 && pr.d != 128) return BSA_ERR_UNSUPPORTED;
+    if (pr.block != 64 && pr.block != 128) return BSA_ERR_UNSUPPORTED;
+    if (pr.score_mode != BSA_SCORE_MEANPOOL && pr.score_mode != BSA_SCORE_PARK) return BSA_ERR_ARG;
+    if (pr.heads < 1 || pr.T < 1 || pr.H < 1 || pr.W < 1 || pr.text_tokens < 0) return BSA_ERR_ARG;
+    const long long nv = (long long)pr.T * pr.H * pr.W;
+    if (nv + pr.text_tokens != (long long)pr.tokens) return BSA_ERR_ARG;
+    if ((long long)pr.heads * pr.tokens * pr.d >= (1LL << 40)) return BSA_ERR_UNSUPPORTED;
+    if (pr.tokens >= (1 << 30)) return BSA_ERR_UNSUPPORTED;
+    int tt, th, tw;
+    const int rc = resolve_tile(pr, &tt, &th, &tw);
+    if (rc != BSA_OK) return rc;
+    Geom x;
+    x.heads = pr.heads;
+    x.N = pr.tokens;
+    x.d = pr.d;
+    x.B = pr.block;
+    x.T = pr.T;
+    x.H = pr.H;
+    x.W = pr.W;
+    x.text = pr.text_tokens;
+    x.tt = tt;
+    x.th = th;
+    x.tw = tw;
+    x.Nv = (int)nv;
+    x.nbv = (int)((nv + pr.block - 1) / pr.block);
+    x.nbt = (pr.text_tokens + pr.block - 1) / pr.block;
+    x.nb = x.nbv + x.nbt;
+    x.slab = (long long)tt * pr.H * pr.W;
+    if (x.nb > kMaxBlocks) return BSA_ERR_UNSUPPORTED;
+    *g = x;
+    return BSA_OK;
+}
+
+size_t pooled_bytes(const Geom& g) { return (size_t)2 * g.heads * g.nb * g.d * sizeof(float); }
+
+int drift_chunks(const Geom& g) {
+    const long long elems = (long long)g.N * g.d;
+    return (int)((elems + kDriftChunkElems - 1) / kDriftChunkElems);
+}
+
+int text_splits(const Geom& g) { return (g.nb + attn::kTextChunk - 1) / attn::kTextChunk; }
+
+size_t attention_ws_bytes(const Geom& g) {
+    if (g.nbt == 0) return 0;
+    const size_t items = (size_t)g.heads * g.nbt * text_splits(g);
+    return items * attn::BQ * (size_t)(g.d + 1) * sizeof(float);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+int launch_status() { return cuda_status(cudaGetLastError()); }
+
+template <int D, int BK>
+int launch_attention(const attn::Params& P, int items, cudaStream_t st) {
+    using C = attn::Cfg<D, BK>;
+    // set on every call: the attribute is per device and the call is cheap
+    if (cudaFuncSetAttribute(attn::sparse_attention_kernel<D, BK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    attn::sparse_attention_kernel<D, BK><<<items, attn::kThreads, C::SMEM, st>>>(P);
+    int rc = launch_status();
+    if (rc != BSA_OK) return rc;
+    if (P.n_text_items > 0) {
+        dim3 grid(P.g.heads * P.g.nbt, attn::BQ);
+        attn::merge_text_kernel<D><<<grid, D, 0, st>>>(P);
+        rc = launch_status();
+    }
+    return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
+    if (out == nullptr) return BSA_ERR_ARG;
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    bsa_plan_info info;
+    std::memset(&info, 0, sizeof(info));
+    info.nb = g.nb;
+    info.nb_video = g.nbv;
+    info.nb_text = g.nbt;
+    info.npad = g.nb * g.B;
+    info.tile_t = g.tt;
+    info.tile_h = g.th;
+    info.tile_w = g.tw;
+    info.score_workspace_bytes = pooled_bytes(g);
+    info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
+    info.attention_workspace_bytes = attention_ws_bytes(g);
+    *out = info;
+    return BSA_OK;
+}
+
+int bsa_block_layout(const bsa_problem* prob, int* perm_host) {
+    if (perm_host == nullptr) return BSA_ERR_ARG;
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    for (int s = 0; s < g.nb * g.B; ++s) perm_host[s] = slot_to_token(g, s);
+    return BSA_OK;
+}
+
+int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                     const int* head_mask, float* scores, void* ws, size_t ws_bytes,
+                     bsa_stream_t stream) {
+    Geom g;
+    int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || scores == nullptr) return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
+    if (ws == nullptr || ws_bytes < pooled_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float* qbar = static_cast<float*>(ws);
+    float* kbar = qbar + (size_t)g.heads * g.nb * g.d;
+    const dim3 pgrid(g.nb, g.heads);
+    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
+    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
+    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
+    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    const float scale = 1.0f / std::sqrt((float)g.d);
+    if (prob->score_mode == BSA_SCORE_MEANPOOL) {
+        const int nbp = (g.nb + 3) & ~3;
+        const bool wide = g.nb > 1024;
+        const int R = wide ? 16 : 32;
+        const size_t smem = (size_t)(R * g.d + R * nbp) * sizeof(float);
+        const dim3 grid((g.nb + R - 1) / R, g.heads);
+#define BSA_MP(DD, RR)                                                                             \
+    do {                                                                                           \
+        if (cudaFuncSetAttribute(meanpool_score_kernel<DD, RR>,                                    \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+            return BSA_ERR_CUDA;                                                                   \
+        meanpool_score_kernel<DD, RR><<<grid, 256, smem, st>>>(g, qbar, kbar, head_mask, scores, scale); \
+    } while (0)
+        if (g.d == 128) { if (wide) BSA_MP(128, 16); else BSA_MP(128, 32); }
+        else { if (wide) BSA_MP(64, 16); else BSA_MP(64, 32); }
+#undef BSA_MP
+        return launch_status();
+    }
+    return launch_park(g, Q, kbar, head_mask, scores, st);
+}
+
+int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p,
+                    const int* head_mask, int* idx, int* cnt, bsa_stream_t stream) {
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (scores == nullptr || p == nullptr || idx == nullptr || cnt == nullptr) return BSA_ERR_ARG;
+    if (!aligned16(scores) || !aligned16(idx) || !aligned16(cnt) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(g.nb, g.heads);
+    if (g.nb <= 64) select_topp_kernel<64><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    else if (g.nb <= 128) select_topp_kernel<128><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    else if (g.nb <= 256) select_topp_kernel<256><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    else if (g.nb <= 512) select_topp_kernel<512><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    else if (g.nb <= 1024) select_topp_kernel<1024><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    else select_topp_kernel<2048><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    return launch_status();
+}
+
+int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                    bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all, float* drift,
+                    int* refresh, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || Q_ref == nullptr || K_ref == nullptr || drift == nullptr ||
+        refresh == nullptr)
+        return BSA_ERR_ARG;
+    if (!(tau >= 0.0f) || std::isinf(tau)) return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(Q_ref) || !aligned16(K_ref) || !aligned16(drift) ||
+        !aligned16(refresh))
+        return BSA_ERR_ALIGN;
+    const int chunks = drift_chunks(g);
+    const size_t need = (size_t)g.heads * chunks * 4 * sizeof(double);
+    if (ws == nullptr || ws_bytes < need) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long long elems = (long long)g.N * g.d;
+    const dim3 grid(chunks, g.heads);
+    double* part = static_cast<double*>(ws);
+    drift_partial_kernel<<<grid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, part);
+    int r2 = launch_status();
+    if (r2 != BSA_OK) return r2;
+    drift_finalize_kernel<<<grid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, tau,
+                                                         part, drift, refresh);
+    return launch_status();
+}
+
+int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                         const bsa_bf16* V, const int* idx, const int* cnt, bsa_bf16* O, void* ws,
+                         size_t ws_bytes, bsa_stream_t stream) {
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || V == nullptr || idx == nullptr || cnt == nullptr || O == nullptr)
+        return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(cnt) || !aligned16(O))
+        return BSA_ERR_ALIGN;
+    const size_t need = attention_ws_bytes(g);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return BSA_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(ws)) return BSA_ERR_ALIGN;
+    attn::Params P;
+    P.g = g;
+    P.Q = Q;
+    P.K = K;
+    P.V = V;
+    P.idx = idx;
+    P.cnt = cnt;
+    P.O = O;
+    P.nsplit = g.nbt > 0 ? text_splits(g) : 1;
+    P.n_text_items = g.heads * g.nbt * (g.nbt > 0 ? P.nsplit : 0);
+    P.part_o = need > 0 ? static_cast<float*>(ws) : nullptr;
+    P.part_lse = need > 0 ? P.part_o + (size_t)P.n_text_items * attn::BQ * g.d : nullptr;
+    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+    const int items = P.n_text_items + g.heads * g.nbv;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (g.d == 128 && g.B == 128) return launch_attention<128, 128>(P, items, st);
+    if (g.d == 128) return launch_attention<128, 64>(P, items, st);
+    if (g.B == 128) return launch_attention<64, 128>(P, items, st);
+    return launch_attention<64, 64>(P, items, st);
+}
+
+int bsa_device_status(bsa_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+    }
+    return word;
+}
+
+const char* bsa_error_string(int status) {
+    switch (status) {
+        case BSA_OK: return "ok";
+        case BSA_ERR_ARG: return "invalid argument";
+        case BSA_ERR_UNSUPPORTED: return "unsupported size (d and block must be 64 or 128; at most 2048 blocks)";
+        case BSA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case BSA_ERR_WORKSPACE: return "workspace missing or too small";
+        case BSA_ERR_CUDA: return "CUDA launch or runtime error";
+        case BSA_ERR_TIMEOUT: return "device: a bounded wait in a kernel ran out";
+        case BSA_ERR_DEVICE_ARG: return "device: kept-block index or count out of range";
+        default: return "unknown status";
+    }
+}
+
+const char* bsa_version(void) { return "bsa 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+// Block pooling and the mean-pooled block scorer.
+//
+// pool_kernel:  qbar[h][i] = mean of Q over the real tokens of block i (same for K).
+//   HBM-bound: every real row of Q and K is read exactly once, 16-byte loads, CD/8 lanes
+//   per 2*d-byte row, float32 accumulation, shared-memory tree reduction.
+// meanpool_score_kernel: S[h][i][j] = softmax_j(qbar_i . kbar_j / sqrt(d)) for 16 or 32
+//   query rows per CTA against every key block; register-blocked float32 dot products,
+//   row softmax in shared memory.
+// (PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers,
+// Abstract: block retrieval from the averaged representations of query and key blocks.)
+#pragma once
+
+#include "bsa_common.cuh"
+
+namespace bsa {
+
+template <int D>
+__device__ inline void accum_bf16x8(float (&acc)[8], const uint4& v) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float2 f = __bfloat1622float2(p[k]);
+        acc[2 * k] += f.x;
+        acc[2 * k + 1] += f.y;
+    }
+}
+
+// grid (nb, heads), 256 threads. Pools Q and K of block i, head h into qbar/kbar [heads][nb][D].
+template <int D, int B>
+__global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __restrict__ Q,
+                                                   const bsa_bf16* __restrict__ K,
+                                                   const int* __restrict__ head_mask,
+                                                   float* __restrict__ qbar, float* __restrict__ kbar) {
+    constexpr int CH = D / 8;               // 16-byte chunks per row
+    constexpr int RPP = 256 / CH;           // rows per pass
+    constexpr int NIT = B / RPP;            // passes
+    const int i = blockIdx.x, h = blockIdx.y;
+    if (head_mask != nullptr && head_mask[h] == 0) return;
+    const int c = threadIdx.x % CH, rs = threadIdx.x / CH;
+    const size_t head_off = (size_t)h * g.N * D;
+
+    int tok[NIT];
+#pragma unroll
+    for (int k = 0; k < NIT; ++k) tok[k] = slot_to_token(g, i * B + rs + k * RPP);
+    uint4 vq[NIT], vk[NIT];
+#pragma unroll
+    for (int k = 0; k < NIT; ++k) {
+        if (tok[k] >= 0) {
+            const size_t off = head_off + (size_t)tok[k] * D + c * 8;
+            vq[k] = __ldg(reinterpret_cast<const uint4*>(Q + off));
+            vk[k] = __ldg(reinterpret_cast<const uint4*>(K + off));
+        } else {
+            vq[k] = make_uint4(0, 0, 0, 0);
+            vk[k] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int k = 0; k < NIT; ++k) {
+        accum_bf16x8<D>(aq, vq[k]);
+        accum_bf16x8<D>(ak, vk[k]);
+    }
+    __shared__ float red[2][RPP][D + 4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        red[0][rs][c * 8 + e] = aq[e];
+        red[1][rs][c * 8 + e] = ak[e];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * D) {
+        const int which = threadIdx.x / D, col = threadIdx.x % D;
+        float s = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < RPP; ++r) s += red[which][r][col];
+        const float n = (float)block_count(g, i);
+        float* out = which == 0 ? qbar : kbar;
+        out[((size_t)h * g.nb + i) * D + col] = s / n;
+    }
+}
+
+// grid (ceil(nb/R), heads), 256 threads; dynamic smem = (R*D + R*nbp) floats.
+// Rows i0..i0+R-1 of head h: logits against every key block, then row softmax.
+template <int D, int R>
+__global__ void __launch_bounds__(256) meanpool_score_kernel(Geom g, const float* __restrict__ qbar,
+                                                             const float* __restrict__ kbar,
+                                                             const int* __restrict__ head_mask,
+                                                             float* __restrict__ scores, float scale) {
+    extern __shared__ float4 smem_f4[];
+    const int h = blockIdx.y, i0 = blockIdx.x * R;
+    if (head_mask != nullptr && head_mask[h] == 0) return;
+    const int nb = g.nb;
+    const int nbp = (nb + 3) & ~3;
+    float* sq = reinterpret_cast<float*>(smem_f4);      // [R][D]
+    float* slog = sq + R * D;                            // [R][nbp]
+    const float* qh = qbar + (size_t)h * nb * D;
+    const float* kh = kbar + (size_t)h * nb * D;
+    for (int e = threadIdx.x; e < R * D; e += 256) {
+        const int r = e / D;
+        sq[e] = (i0 + r < nb) ? qh[(size_t)(i0 + r) * D + (e % D)] : 0.f;
+    }
+    __syncthreads();
+    const float4* sq4 = reinterpret_cast<const float4*>(sq);
+    for (int jb = 0; jb < nb; jb += 512) {
+        const int ja = jb + threadIdx.x, jbb = ja + 256;
+        const float4* ka = reinterpret_cast<const float4*>(kh + (size_t)min(ja, nb - 1) * D);
+        const float4* kb = reinterpret_cast<const float4*>(kh + (size_t)min(jbb, nb - 1) * D);
+        float acc0[R], acc1[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) { acc0[r] = 0.f; acc1[r] = 0.f; }
+#pragma unroll 2
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+            const float4 a = __ldg(ka + c4), b = __ldg(kb + c4);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float4 q = sq4[r * (D / 4) + c4];
+                acc0[r] = fmaf(q.x, a.x, acc0[r]);
+                acc0[r] = fmaf(q.y, a.y, acc0[r]);
+                acc0[r] = fmaf(q.z, a.z, acc0[r]);
+                acc0[r] = fmaf(q.w, a.w, acc0[r]);
+                acc1[r] = fmaf(q.x, b.x, acc1[r]);
+                acc1[r] = fmaf(q.y, b.y, acc1[r]);
+                acc1[r] = fmaf(q.z, b.z, acc1[r]);
+                acc1[r] = fmaf(q.w, b.w, acc1[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (ja < nb) slog[r * nbp + ja] = acc0[r] * scale;
+            if (jbb < nb) slog[r * nbp + jbb] = acc1[r] * scale;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int r = warp; r < R; r += 8) {
+        if (i0 + r >= nb) break;
+        float* row = slog + r * nbp;
+        float mx = -INFINITY;
+        for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, row[j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+        for (int j = lane; j < nb; j += 32) {
+            const float e = expf(row[j] - mx);
+            row[j] = e;
+            sum += e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = 1.0f / sum;
+        float* out = scores + ((size_t)h * nb + i0 + r) * nb;
+        for (int j = lane; j < nb; j += 32) out[j] = row[j] * inv;
+    }
+}
+
+}  // namespace bsa

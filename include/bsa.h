@@ -1,0 +1,176 @@
+/*
+ * bsa.h — C ABI of libbsa: training-free block-sparse 3D attention for video diffusion
+ * transformers on NVIDIA B200 (sm_100a).
+ *
+ * One attention layer's hot path, per denoising step:
+ *   bsa_drift_check      per-head query/key drift against the cached reference; decides
+ *                        which heads refresh their mask (HEART: Exploiting Head
+ *                        Heterogeneity in Sparse Attention for Video Diffusion, abstract,
+ *                        "Temporal Mask Reuse"; HASTE, abstract)
+ *   bsa_score_blocks     query-block x key-block importance, mean-pooled or per-query
+ *                        normalised (PARK: Accurate Block Retrieval for Sparse Attention in
+ *                        Video Diffusion Transformers, Abstract)
+ *   bsa_select_topp      per-head top-p kept-block lists (HASTE: Training-Free Video
+ *                        Diffusion Acceleration via Head-Wise Adaptive Sparse Attention,
+ *                        abstract)
+ *   bsa_sparse_attention softmax attention over the kept key blocks only (PARK, Abstract:
+ *                        attention computed only within the retrieved blocks)
+ *
+ * Conventions shared by every call
+ *   - Tensors Q, K, V, O are bfloat16 (raw 16-bit patterns, bsa_bf16), row-major
+ *     [heads, tokens, d] in RASTER order of the 3D grid (t slowest, x fastest), video tokens
+ *     first, then `text_tokens` text tokens. The library never permutes them in memory: the
+ *     kernels gather rows in block order on the fly.
+ *   - Block order: the video grid is cut into tiles (tile_t x tile_h x tile_w) visited in
+ *     raster order of tile coordinates; tokens inside a tile are in raster order and edge
+ *     tiles are truncated. That concatenated order is cut into blocks of `block` tokens; only
+ *     the last video block can be partial (its missing slots are padding, masked as keys and
+ *     never written as queries). Text tokens follow as their own blocks (nb_text of them).
+ *     nb = nb_video + nb_text blocks per head.
+ *   - All pointers are DEVICE pointers to caller-owned memory, 16-byte aligned, unless a
+ *     parameter says "host". The library allocates and frees nothing; scratch comes from the
+ *     caller's workspace, sized by bsa_plan.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and returns a status code. Argument errors are detected on the host before anything is
+ *     launched; nothing is written then. Device-side problems (a bounded wait that ran out, an
+ *     out-of-range kept-block index) set a device error word read by bsa_device_status.
+ *   - Thread safety: calls only read their arguments; concurrent calls on different streams
+ *     are safe as long as their output buffers and workspaces do not overlap.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t bsa_bf16;                 /* bfloat16 bit pattern */
+typedef struct CUstream_st* bsa_stream_t;  /* identical to cudaStream_t */
+
+/* status codes */
+#define BSA_OK               0
+#define BSA_ERR_ARG         -1   /* null pointer, bad size, inconsistent problem */
+#define BSA_ERR_UNSUPPORTED -2   /* d or block outside the supported set */
+#define BSA_ERR_ALIGN       -3   /* a pointer is not 16-byte aligned */
+#define BSA_ERR_WORKSPACE   -4   /* workspace missing or smaller than bsa_plan asks */
+#define BSA_ERR_CUDA        -5   /* a CUDA launch or runtime call failed */
+#define BSA_ERR_TIMEOUT     -6   /* device: a bounded wait inside a kernel ran out */
+#define BSA_ERR_DEVICE_ARG  -7   /* device: a kept-block index or count was out of range */
+
+/* scorers (PARK, Abstract) */
+#define BSA_SCORE_MEANPOOL   0   /* softmax_j( mean(Q in block i) . mean(K in block j) / sqrt(d) ) */
+#define BSA_SCORE_PARK       1   /* mean over real q in block i of softmax_j( q . mean(K in block j) / sqrt(d) ) */
+
+/* One attention layer. Plain struct, passed by pointer, read only. */
+typedef struct bsa_problem {
+    int heads;          /* >= 1 */
+    int tokens;         /* must equal T*H*W + text_tokens */
+    int d;              /* head dimension: 64 or 128 */
+    int T, H, W;        /* 3D video grid, each >= 1 */
+    int text_tokens;    /* >= 0, appended after the video tokens */
+    int block;          /* tokens per block: 64 or 128 */
+    int tile_t, tile_h, tile_w;  /* tile shape; all 0 = default (1x8x8 for 64, 2x8x8 for 128);
+                                    otherwise tile_t*tile_h*tile_w must equal block */
+    int score_mode;     /* BSA_SCORE_MEANPOOL or BSA_SCORE_PARK */
+} bsa_problem;
+
+/* Derived sizes, filled by bsa_plan (host only, no CUDA call). */
+typedef struct bsa_plan_info {
+    int nb;             /* blocks per head = nb_video + nb_text */
+    int nb_video;       /* ceil(T*H*W / block) */
+    int nb_text;        /* ceil(text_tokens / block) */
+    int npad;           /* nb * block */
+    int tile_t, tile_h, tile_w;  /* tile actually used */
+    size_t score_workspace_bytes;      /* bsa_score_blocks */
+    size_t drift_workspace_bytes;      /* bsa_drift_check */
+    size_t attention_workspace_bytes;  /* bsa_sparse_attention */
+} bsa_plan_info;
+
+/* Validate `prob` and fill `out`. Host only; launches nothing.
+ * Returns BSA_OK, BSA_ERR_ARG or BSA_ERR_UNSUPPORTED. */
+int bsa_plan(const bsa_problem* prob, bsa_plan_info* out);
+
+/* Block layout on the host: perm_host[s] = raster token index held by block slot s, or -1
+ * for a padding slot, for s in [0, plan.npad). Host memory, caller-owned, plan.npad ints.
+ * Host only (the kernels compute the same map on the fly). Returns BSA_OK or BSA_ERR_ARG. */
+int bsa_block_layout(const bsa_problem* prob, int* perm_host);
+
+/* Block importance scores (PARK, Abstract: retrieval from averaged query/key block
+ * representations, and PARK's per-query normalisation averaged within the query block).
+ *   Q, K       [heads, tokens, d] bf16, raster order.
+ *   head_mask  [heads] int, device, nullable. Heads with head_mask[h] == 0 are skipped and
+ *              their rows of `scores` are left untouched (the cached-mask case).
+ *   scores     [heads, nb, nb] float32 out. Row (h, i) is a probability distribution over
+ *              key blocks j (including text blocks); logits are scaled by 1/sqrt(d).
+ *   ws         workspace of at least plan.score_workspace_bytes (pooled block means).
+ * Mode is prob->score_mode. */
+int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                     const int* head_mask, float* scores,
+                     void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Per-head top-p kept-block lists (HASTE, abstract: online top-p with per-head thresholds).
+ * For each row (h, i): key blocks ordered by score descending, then index ascending; the
+ * shortest prefix whose float32 cumulative score reaches p[h] (>=) is kept (at least one
+ * block; p[h] >= 1 keeps all). Video query rows additionally keep every text key block; text
+ * query rows keep every block. The kept list is written in that same order.
+ *   scores     [heads, nb, nb] float32 (from bsa_score_blocks).
+ *   p          [heads] float32, device.
+ *   head_mask  [heads] int, device, nullable: heads with 0 are skipped (idx/cnt untouched).
+ *   idx        [heads, nb, nb] int32 out: idx[h][i][0..cnt-1] are kept block indices;
+ *              entries at and after cnt are not written.
+ *   cnt        [heads, nb] int32 out, 1 <= cnt <= nb. */
+int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p,
+                    const int* head_mask, int* idx, int* cnt, bsa_stream_t stream);
+
+/* Temporal mask reuse gate (HEART, abstract: refresh a head's cached mask only when its
+ * query-key drift exceeds a prescribed threshold).
+ *   drift[h]   = max(||Q_h - Qref_h||_F / ||Qref_h||_F, ||K_h - Kref_h||_F / ||Kref_h||_F)
+ *                over all tokens of head h (0 when both norms are 0; +inf when only the
+ *                reference norm is 0).
+ *   refresh[h] = force_all || drift[h] > tau.
+ * For every refreshed head the call then copies Q_h -> Q_ref_h and K_h -> K_ref_h (the new
+ * reference), after the decision is made. Pass force_all = 1 on the first step, when there is
+ * no reference yet (Q_ref/K_ref may then hold anything finite or not).
+ *   Q, K           [heads, tokens, d] bf16, current step.
+ *   Q_ref, K_ref   [heads, tokens, d] bf16, in/out reference snapshots.
+ *   drift          [heads] float32 out;  refresh [heads] int32 out (0/1; usable as head_mask).
+ *   ws             at least plan.drift_workspace_bytes. The reduction order is fixed, so the
+ *                  result is deterministic. */
+int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                    bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all,
+                    float* drift, int* refresh,
+                    void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Block-sparse attention (PARK, Abstract: attention computed only within the retrieved
+ * blocks). For every real query t of query block i of head h:
+ *   O_t = sum over the real keys u of blocks idx[h][i][0..cnt[h][i]-1] of
+ *         softmax_u(Q_t . K_u / sqrt(d)) V_u
+ * bf16 inputs, float32 accumulation and softmax, bf16 output.
+ *   Q, K, V    [heads, tokens, d] bf16, raster order.
+ *   idx, cnt   as written by bsa_select_topp (any lists with 1 <= cnt <= nb and distinct
+ *              indices in [0, nb) are accepted; a bad entry sets BSA_ERR_DEVICE_ARG in the
+ *              device error word and the row's output is unspecified).
+ *   O          [heads, tokens, d] bf16 out, raster order. Every real token is written.
+ *   ws         at least plan.attention_workspace_bytes (partial results of the dense text
+ *              rows, which are split across CTAs). */
+int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                         const bsa_bf16* V, const int* idx, const int* cnt, bsa_bf16* O,
+                         void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device.
+ * Returns BSA_OK, BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_ARG or BSA_ERR_CUDA. */
+int bsa_device_status(bsa_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* bsa_error_string(int status);
+
+/* Library version, e.g. "bsa 0.1.0 sm_100a". */
+const char* bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */

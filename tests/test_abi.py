@@ -1,0 +1,107 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol include/bsa.h
+declares, plans sizes, reproduces the oracle's block layout exactly, and rejects bad
+arguments before launching anything."""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_attention_query_b200 import build as bsa_build
+
+bsa_build.build()
+from block_sparse_attention_query_b200 import bsa  # noqa: E402
+from block_sparse_attention_query_b200 import inputs  # noqa: E402
+from oracle import bsa_oracle as O  # noqa: E402
+from tests.conftest import GOLDEN, ROOT  # noqa: E402
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "bsa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(bsa_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared_symbols()
+    assert "bsa_sparse_attention" in names and len(names) >= 9
+    for n in names:
+        assert hasattr(bsa.lib, n), n
+        assert n in bsa.EXPORTS, n
+
+
+def test_version_and_error_strings():
+    assert "sm_100a" in bsa.bsa_version()
+    for code in range(-7, 1):
+        assert bsa.lib.bsa_error_string(code)
+    assert bsa.lib.bsa_error_string(-99) == b"unknown status"
+
+
+@pytest.mark.parametrize("name", inputs.WORKLOADS)
+def test_plan_matches_oracle_layout(name):
+    w = inputs.workload(name)
+    prob = bsa.problem(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block)
+    info = bsa.bsa_plan(prob)
+    L = O.block_layout(w.T, w.H, w.W, w.text_tokens, w.block)
+    assert (info.nb, info.nb_video, info.nb_text, info.npad) == (L.nb, L.nb_video, L.nb_text, L.npad)
+    perm = np.array(bsa.bsa_block_layout(prob))
+    assert np.array_equal(perm, L.perm)
+
+
+def test_block_layout_golden_and_odd_tiles():
+    with open(os.path.join(GOLDEN, "layout_small.json")) as f:
+        cases = json.load(f)["cases"]
+    # the library only accepts blocks of 64/128 tokens: scale the hand cases' grids up by
+    # using tiles whose volume is the block size, and compare against the oracle
+    for T, H, W, text, B, tile in [(3, 5, 7, 0, 64, (1, 8, 8)), (5, 9, 17, 40, 64, (4, 4, 4)),
+                                   (7, 13, 11, 130, 128, (2, 8, 8)), (2, 3, 50, 5, 64, (1, 2, 32)),
+                                   (9, 9, 9, 0, 128, (8, 4, 4))]:
+        prob = bsa.problem(1, 64, T, H, W, text, B, tile)
+        L = O.block_layout(T, H, W, text, B, tile)
+        assert np.array_equal(np.array(bsa.bsa_block_layout(prob)), L.perm)
+    assert len(cases) >= 3
+
+
+def test_plan_rejects_bad_problems():
+    good = bsa.problem(2, 64, 4, 16, 16, 0, 64)
+    info = bsa.PlanInfo()
+    assert bsa.lib.bsa_plan(ctypes.byref(good), ctypes.byref(info)) == bsa.BSA_OK
+    bad = []
+    p = bsa.problem(2, 96, 4, 16, 16, 0, 64); bad.append((p, bsa.BSA_ERR_UNSUPPORTED))
+    p = bsa.problem(2, 64, 4, 16, 16, 0, 32); bad.append((p, bsa.BSA_ERR_UNSUPPORTED))
+    p = bsa.problem(2, 64, 4, 16, 16, 0, 64); p.tokens += 1; bad.append((p, bsa.BSA_ERR_ARG))
+    p = bsa.problem(0, 64, 4, 16, 16, 0, 64); bad.append((p, bsa.BSA_ERR_ARG))
+    p = bsa.problem(2, 64, 4, 16, 16, 0, 64, tile=(2, 8, 8)); bad.append((p, bsa.BSA_ERR_ARG))
+    p = bsa.problem(2, 64, 4, 16, 16, 0, 64, score_mode=7); bad.append((p, bsa.BSA_ERR_ARG))
+    p = bsa.problem(2, 64, 64, 64, 64, 0, 64); bad.append((p, bsa.BSA_ERR_UNSUPPORTED))  # 4096 blocks
+    for prob, code in bad:
+        assert bsa.lib.bsa_plan(ctypes.byref(prob), ctypes.byref(info)) == code
+    assert bsa.lib.bsa_plan(None, ctypes.byref(info)) == bsa.BSA_ERR_ARG
+    assert bsa.lib.bsa_plan(ctypes.byref(good), None) == bsa.BSA_ERR_ARG
+
+
+def test_calls_reject_bad_pointers_before_launch():
+    # host-side validation only: no pointer is dereferenced and nothing is launched
+    prob = bsa.problem(2, 64, 4, 16, 16, 0, 64)
+    L = bsa.lib
+    a = ctypes.c_void_p(4096)          # aligned, never dereferenced on these paths
+    mis = ctypes.c_void_p(4096 + 2)
+    pr = ctypes.byref(prob)
+    assert L.bsa_score_blocks(pr, None, a, None, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_score_blocks(pr, mis, a, None, a, a, 1 << 20, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_score_blocks(pr, a, a, None, a, a, 16, None) == bsa.BSA_ERR_WORKSPACE
+    assert L.bsa_score_blocks(pr, a, a, None, a, None, 1 << 20, None) == bsa.BSA_ERR_WORKSPACE
+    assert L.bsa_select_topp(pr, a, None, None, a, a, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_select_topp(pr, a, a, mis, a, a, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(-1.0), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(float("nan")), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(0.05), 0, a, a, a, 8, None) == bsa.BSA_ERR_WORKSPACE
+    assert L.bsa_drift_check(pr, a, a, a, None, ctypes.c_float(0.05), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_sparse_attention(pr, a, a, a, a, a, None, a, 0, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_sparse_attention(pr, a, a, mis, a, a, a, a, 0, None) == bsa.BSA_ERR_ALIGN
+    text = bsa.problem(2, 64, 4, 16, 16, 64, 64)
+    need = bsa.bsa_plan(text).attention_workspace_bytes
+    assert need > 0
+    assert L.bsa_sparse_attention(ctypes.byref(text), a, a, a, a, a, a, a, need - 1, None) == bsa.BSA_ERR_WORKSPACE

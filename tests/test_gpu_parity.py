@@ -1,0 +1,355 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs, call by call, through the C ABI.
+
+Tolerances (stated by the task's parity rule for bf16 inputs with fp32 accumulation):
+attention max-abs <= 3e-2 and relative-L2 <= 1e-2 on the oracle's mask; kept lists
+bit-exact except rows the comparison rule in tests/parity.py exempts; scores within the
+float32 error bound of the scorer."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_query_b200 import inputs
+from oracle import bsa_oracle as O
+from tests import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+ATT_MAX_ABS = 3e-2
+ATT_REL_L2 = 1e-2
+SCORE_RTOL = 5e-5      # float32 scorer vs float64 oracle, relative (see parity.TIE_REL)
+SCORE_ATOL = 1e-7
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_attention_query_b200 import build
+    build.build()
+
+
+def _bsa():
+    from block_sparse_attention_query_b200 import bsa
+    return bsa
+
+
+class Case:
+    """Inputs on host and device plus the problem descriptor."""
+
+    def __init__(self, heads, d, T, H, W, text, B, p, mode="meanpool", seed=0, tile=(0, 0, 0)):
+        bsa = _bsa()
+        self.heads, self.d, self.B = heads, d, B
+        self.Qb, self.Kb, self.Vb = inputs.generate_qkv(heads, d, T, H, W, text, seed)
+        self.N = self.Qb.shape[1]
+        self.p = np.array([p] * heads if np.isscalar(p) else p, dtype=np.float64)
+        self.mode = mode
+        smode = bsa.BSA_SCORE_PARK if mode == "park" else bsa.BSA_SCORE_MEANPOOL
+        self.prob = bsa.problem(heads, d, T, H, W, text, B, tile, smode)
+        self.plan = bsa.bsa_plan(self.prob)
+        self.layout = O.block_layout(T, H, W, text, B, tile if tile != (0, 0, 0) else None)
+        self.Q, self.K, self.V = (PT.to_dev_bf16(x) for x in (self.Qb, self.Kb, self.Vb))
+        nb = self.plan.nb
+        self.nb = nb
+        self.p_dev = torch.tensor(self.p, dtype=torch.float32, device="cuda")
+
+    def ws(self, nbytes):
+        return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device="cuda")
+
+    def gpu_scores(self):
+        bsa = _bsa()
+        S = torch.empty(self.heads, self.nb, self.nb, dtype=torch.float32, device="cuda")
+        bsa.bsa_score_blocks(self.prob, self.Q, self.K, None, S, self.ws(self.plan.score_workspace_bytes))
+        return S
+
+    def gpu_select(self, S):
+        bsa = _bsa()
+        idx = torch.full((self.heads, self.nb, self.nb), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(self.heads, self.nb, dtype=torch.int32, device="cuda")
+        bsa.bsa_select_topp(self.prob, S, self.p_dev, None, idx, cnt)
+        return idx, cnt
+
+    def gpu_attention(self, idx, cnt):
+        bsa = _bsa()
+        Od = torch.full((self.heads, self.N, self.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        bsa.bsa_sparse_attention(self.prob, self.Q, self.K, self.V, idx, cnt, Od,
+                                 self.ws(self.plan.attention_workspace_bytes))
+        return Od
+
+    def oracle_scores(self, h):
+        return O.score_head(O.bf16_to_f64(self.Qb[h]), O.bf16_to_f64(self.Kb[h]), self.layout, self.mode)
+
+
+def _status_ok():
+    assert _bsa().bsa_device_status() == 0
+
+
+SMALL = {
+    "tiny": dict(heads=2, d=64, T=4, H=16, W=16, text=0, B=64, p=0.9),
+    # ragged last block with a single real token, d=128 with 64-token blocks
+    "ragged_d128_b64": dict(heads=2, d=128, T=3, H=9, W=19, text=0, B=64, p=0.85),
+    # text blocks (one partial), d=64 with 128-token blocks, odd grid
+    "text_d64_b128": dict(heads=3, d=64, T=5, H=11, W=13, text=200, B=128, p=0.9),
+    # d=128, B=128 with text, several tiles and a partial last video block
+    "text_d128_b128": dict(heads=2, d=128, T=6, H=20, W=24, text=256, B=128, p=0.95),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("mode", ["meanpool", "park"])
+def test_scores_match_oracle(name, mode):
+    c = Case(**SMALL[name], mode=mode)
+    S = c.gpu_scores().cpu().numpy()
+    torch.cuda.synchronize()
+    _status_ok()
+    for h in range(c.heads):
+        ref = c.oracle_scores(h)
+        err = np.abs(S[h] - ref)
+        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * ref), (h, float(err.max()))
+        assert np.allclose(S[h].sum(axis=1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_select_on_oracle_scores_is_exact(name):
+    # same float32 scores on both sides: only the cumulative-sum rounding may differ
+    c = Case(**SMALL[name])
+    S = np.stack([c.oracle_scores(h).astype(np.float32) for h in range(c.heads)])
+    idx, cnt = c.gpu_select(torch.from_numpy(S).cuda())
+    _status_ok()
+    res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, c.p, c.layout)
+    assert res["mismatch"] == 0 and res["tie"] == 0, res
+    assert res["exact"] >= (c.heads * c.nb) - 2, res
+
+
+@pytest.mark.parametrize("p", [1.0, 1e-6, 0.5])
+def test_select_edge_p(p):
+    c = Case(**{**SMALL["text_d64_b128"], "p": p})
+    S = np.stack([c.oracle_scores(h).astype(np.float32) for h in range(c.heads)])
+    idx, cnt = c.gpu_select(torch.from_numpy(S).cuda())
+    cnt = cnt.cpu().numpy()
+    if p == 1.0:
+        assert (cnt == c.nb).all()
+    if p == 1e-6:
+        assert (cnt[:, :c.layout.nb_video] == 1 + c.layout.nb_text).all()
+    res = PT.compare_masks(idx.cpu().numpy(), cnt, S, c.p, c.layout)
+    assert res["mismatch"] == 0 and res["tie"] == 0, res
+
+
+def test_select_hand_rows():
+    # the hand-derived rows of tests/golden/topp_cases.json, padded into one head of 64 blocks
+    import json, os
+    from tests.conftest import GOLDEN
+    bsa = _bsa()
+    with open(os.path.join(GOLDEN, "topp_cases.json")) as f:
+        cases = [c for c in json.load(f)["cases"] if not c["forced"]]
+    prob = bsa.problem(1, 64, 1, 64, 64, 0, 64)       # 64 blocks, no text
+    nb = bsa.bsa_plan(prob).nb
+    for c in cases:
+        row = np.zeros(nb, np.float32)
+        row[:len(c["scores"])] = c["scores"]
+        S = torch.from_numpy(np.tile(row, (nb, 1))[None]).cuda().contiguous()
+        pd = torch.tensor([c["p"]], dtype=torch.float32, device="cuda")
+        idx = torch.full((1, nb, nb), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(1, nb, dtype=torch.int32, device="cuda")
+        bsa.bsa_select_topp(prob, S, pd, None, idx, cnt)
+        n = cnt[0, 0].item()
+        got = idx[0, 0, :n].tolist()
+        if c["p"] >= 1.0:
+            assert got[:len(c["kept"])] == c["kept"]
+        else:
+            assert got == c["kept"], c["why"]
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("mode", ["meanpool", "park"])
+def test_masks_end_to_end(name, mode):
+    c = Case(**SMALL[name], mode=mode)
+    idx, cnt = c.gpu_select(c.gpu_scores())
+    _status_ok()
+    S = np.stack([c.oracle_scores(h).astype(np.float32) for h in range(c.heads)])
+    res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, c.p, c.layout)
+    assert res["mismatch"] == 0, res
+
+
+def _oracle_mask(c):
+    idxs, cnts = [], []
+    for h in range(c.heads):
+        S = c.oracle_scores(h).astype(np.float32)
+        i_, c_ = O.select_topp(S, c.p[h], c.layout)
+        idxs.append(i_)
+        cnts.append(c_)
+    return np.stack(idxs), np.stack(cnts)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention_on_oracle_mask(name):
+    c = Case(**SMALL[name])
+    idx, cnt = _oracle_mask(c)
+    Od = c.gpu_attention(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    _status_ok()
+    got = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    for h in range(c.heads):
+        ref = O.sparse_attention_head(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]),
+                                      O.bf16_to_f64(c.Vb[h]), idx[h], cnt[h], c.layout)
+        assert np.isfinite(got[h]).all()
+        mx, rel = PT.attention_errors(got[h], ref, np.arange(c.N))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (h, mx, rel)
+
+
+def test_attention_dense_mask_equals_dense_attention():
+    # p = 1 keeps every block: the sparse kernel must reproduce dense softmax attention
+    c = Case(**{**SMALL["text_d128_b128"], "p": 1.0})
+    idx = np.tile(np.arange(c.nb, dtype=np.int32), (c.heads, c.nb, 1))
+    cnt = np.full((c.heads, c.nb), c.nb, np.int32)
+    Od = c.gpu_attention(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    _status_ok()
+    got = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    for h in range(c.heads):
+        q, k, v = (torch.from_numpy(O.bf16_to_f64(x[h])) for x in (c.Qb, c.Kb, c.Vb))
+        ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0].numpy()
+        mx, rel = PT.attention_errors(got[h], ref, np.arange(c.N))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (h, mx, rel)
+
+
+def test_attention_single_block_rows_and_constant_v():
+    # cnt = 1 everywhere (each row attends its own block); V constant => O constant
+    c = Case(**SMALL["ragged_d128_b64"])
+    c.V = torch.full_like(c.V, 0.375)
+    idx = np.tile(np.arange(c.nb, dtype=np.int32)[:, None], (c.heads, 1, c.nb))
+    cnt = np.ones((c.heads, c.nb), np.int32)
+    Od = c.gpu_attention(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    _status_ok()
+    got = Od.float().cpu().numpy()
+    assert np.all(got == 0.375)
+
+
+def test_attention_bad_index_sets_device_error():
+    # out-of-range kept index and count: the kernel's own checks flag them (no fault)
+    bsa = _bsa()
+    c = Case(**SMALL["tiny"])
+    idx, cnt = _oracle_mask(c)
+    idx[0, 3, 0] = c.nb + 5
+    cnt[1, 2] = c.nb + 1
+    c.gpu_attention(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    assert bsa.bsa_device_status() == bsa.BSA_ERR_DEVICE_ARG
+    assert bsa.bsa_device_status() == 0   # cleared after reading
+
+
+def test_drift_matches_oracle_and_snapshots():
+    bsa = _bsa()
+    c = Case(**SMALL["text_d64_b128"])
+    rng = np.random.default_rng(5)
+    scale = np.array([1.0, 1.03, 1.2])            # per-head drift 0, 0.03, 0.2 on Q
+    Qref_bits = c.Qb.copy()
+    Q2 = inputs.f32_to_bf16_bits((O.bf16_to_f64(c.Qb) * scale[:, None, None]).astype(np.float32))
+    K2 = c.Kb.copy()
+    K2[2, :10] = inputs.f32_to_bf16_bits(rng.standard_normal((10, c.d)).astype(np.float32))
+    Qd, Kd = PT.to_dev_bf16(Q2), PT.to_dev_bf16(K2)
+    Qr, Kr = PT.to_dev_bf16(Qref_bits), PT.to_dev_bf16(c.Kb)
+    drift = torch.zeros(c.heads, dtype=torch.float32, device="cuda")
+    refresh = torch.zeros(c.heads, dtype=torch.int32, device="cuda")
+    bsa.bsa_drift_check(c.prob, Qd, Kd, Qr, Kr, 0.05, 0, drift, refresh, c.ws(c.plan.drift_workspace_bytes))
+    _status_ok()
+    for h in range(c.heads):
+        ref = O.drift(O.bf16_to_f64(Q2[h]), O.bf16_to_f64(K2[h]), O.bf16_to_f64(Qref_bits[h]),
+                      O.bf16_to_f64(c.Kb[h]))
+        assert drift[h].item() == pytest.approx(ref, rel=1e-6, abs=1e-9)
+        assert bool(refresh[h].item()) == (ref > 0.05)
+    # refreshed heads now hold the new snapshot, the others the old one
+    qr, kr = PT.from_dev_bf16(Qr), PT.from_dev_bf16(Kr)
+    for h in range(c.heads):
+        fresh = bool(refresh[h].item())
+        assert np.array_equal(qr[h], Q2[h] if fresh else Qref_bits[h])
+        assert np.array_equal(kr[h], K2[h] if fresh else c.Kb[h])
+    # force_all refreshes everything and snapshots all heads
+    bsa.bsa_drift_check(c.prob, Qd, Kd, Qr, Kr, 0.05, 1, drift, refresh, c.ws(c.plan.drift_workspace_bytes))
+    assert refresh.cpu().tolist() == [1, 1, 1]
+    assert np.array_equal(PT.from_dev_bf16(Qr), Q2) and np.array_equal(PT.from_dev_bf16(Kr), K2)
+    # nothing changed since: zero drift, no refresh
+    bsa.bsa_drift_check(c.prob, Qd, Kd, Qr, Kr, 0.05, 0, drift, refresh, c.ws(c.plan.drift_workspace_bytes))
+    assert refresh.cpu().tolist() == [0, 0, 0]
+    assert drift.cpu().tolist() == [0.0, 0.0, 0.0]
+
+
+def test_reuse_run_tiny_50_steps():
+    """Drift-gated mask reuse over 50 steps on the tiny shape: refresh decisions, kept lists
+    and outputs follow the oracle step by step."""
+    from block_sparse_attention_query_b200.layer import SparseAttentionLayer
+    w = inputs.workload("tiny")
+    walk = inputs.RandomWalk(w.heads, w.d, w.T, w.H, w.W, 0, seed=0)
+    layer = SparseAttentionLayer(w.heads, w.d, w.T, w.H, w.W, 0, w.block, p=0.9, tau=0.05)
+    L = O.block_layout(w.T, w.H, w.W, 0, w.block)
+    Vd = PT.to_dev_bf16(walk.V)
+    Od = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device="cuda")
+    steps = []
+    gpu_flags, gpu_out = [], []
+    for s in range(50):
+        q, k, _ = walk.current()
+        steps.append((q, k))
+        layer.step(PT.to_dev_bf16(q), PT.to_dev_bf16(k), Vd, Od)
+        gpu_flags.append(layer.refresh.cpu().tolist())
+        if s in (0, 17, 49):
+            gpu_out.append(PT.bf16_bits_f64(PT.from_dev_bf16(Od)))
+        walk.advance()
+    _status_ok()
+    ref = O.reuse_run(steps, walk.V, L, [0.9] * w.heads, 0.05)
+    flags_ref = [[int(x) for x in row] for row in ref["refresh"]]
+    for s, (a, b, d) in enumerate(zip(gpu_flags, flags_ref, ref["drift"])):
+        if a != b:  # only a drift within 1e-6 of tau may flip
+            assert all(abs(x - 0.05) <= 1e-6 for x, u, v in zip(d, a, b) if u != v), (s, a, b, d)
+    assert sum(map(sum, gpu_flags)) == sum(map(sum, flags_ref))
+    assert sum(map(sum, flags_ref)) > w.heads       # the walk does trigger refreshes
+    for o, s in zip(gpu_out, (0, 17, 49)):
+        mx, rel = PT.attention_errors(o, ref["O"][s], np.arange(w.tokens))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (s, mx, rel)
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _full_case(name, mode="meanpool"):
+    w = inputs.workload(name)
+    return Case(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, list(w.p), mode=mode)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,mode", [("wan13b_480p", "meanpool"), ("wan13b_480p", "park"),
+                                       ("wan14b_720p", "meanpool"), ("wan14b_720p", "park"),
+                                       ("hunyuan_720p", "meanpool")])
+def test_full_size_masks_and_sampled_attention(name, mode):
+    c = _full_case(name, mode)
+    S_gpu = c.gpu_scores()
+    idx, cnt = c.gpu_select(S_gpu)
+    _status_ok()
+    heads = sorted(set([0, c.heads // 2, c.heads - 1]))
+    S_gpu = S_gpu.cpu().numpy()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    rng = np.random.default_rng(0)
+    S_or = np.zeros_like(S_gpu)
+    for h in heads:
+        S_or[h] = c.oracle_scores(h).astype(np.float32)
+        err = np.abs(S_gpu[h] - S_or[h])
+        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * S_or[h]), (h, float(err.max()))
+    res = PT.compare_masks(idx_h, cnt_h, S_or, c.p, c.layout, heads=heads)
+    assert res["mismatch"] == 0, res
+    # attention on the oracle's mask for sampled query blocks (text rows included)
+    oi = {h: O.select_topp(S_or[h], c.p[h], c.layout) for h in heads}
+    idx_o = idx.clone()
+    cnt_o = cnt.clone()
+    for h in heads:
+        idx_o[h] = torch.from_numpy(oi[h][0]).cuda()
+        cnt_o[h] = torch.from_numpy(oi[h][1]).cuda()
+    Od = c.gpu_attention(idx_o, cnt_o)
+    _status_ok()
+    got = Od.float()
+    for h in heads:
+        qbl = sorted(set(rng.choice(c.layout.nb, 6, replace=False).tolist() + [c.layout.nb - 1]))
+        ref = O.sparse_attention_head(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]),
+                                      O.bf16_to_f64(c.Vb[h]), oi[h][0], oi[h][1], c.layout, qblocks=qbl)
+        rows = np.concatenate([c.layout.rows(i) for i in qbl])
+        mx, rel = PT.attention_errors(got[h].cpu().double().numpy(), ref, rows)
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (h, mx, rel)
+    # properties at full size on every row: finite, and each output is a convex
+    # combination of V rows (bounded by the V range)
+    vmax = float(np.abs(O.bf16_to_f64(c.Vb)).max())
+    assert torch.isfinite(got).all() and float(got.abs().max()) <= vmax + 1e-2
