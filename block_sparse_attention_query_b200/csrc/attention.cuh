@@ -283,8 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
-                if (m_new > m) {
-                    const float alpha = exp2f(m - m_new);
+                // tcgen05.ld/st are warp-collective (.sync.aligned): the rescale runs for the
+                // whole warp when any of its rows saw a larger max (alpha = 1 elsewhere)
+                const bool grow = m_new > m;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float alpha = grow ? exp2f(m - m_new) : 1.0f;
                     l *= alpha;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
@@ -351,8 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 }
             }
             P.part_lse[(size_t)t_item * BQ + r] = (ok && n > 0) ? m + log2f(l) : -INFINITY;
-        } else if (row_real) {
-            bsa_bf16* orow = P.O + head_off + (size_t)q_token * D;
+        } else {
+            // every lane takes part in the warp-collective TMEM loads; only real rows store
+            bsa_bf16* orow = P.O + head_off + (size_t)(row_real ? q_token : 0) * D;
             const float inv = (ok && n > 0) ? 1.0f / l : 0.f;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
@@ -364,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) t[e] = 0u;
                 }
+                if (!row_real) continue;
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint32_t pk[4];
