@@ -66,7 +66,8 @@ int make_geom(const bsa_problem* prob, Geom* g) {
     x.nbv = (int)((nv + pr.block - 1) / pr.block);
     x.nbt = (pr.text_tokens + pr.block - 1) / pr.block;
     x.nb = x.nbv + x.nbt;
-    x.slab = (long long)tt * pr.H * pr.W;
+    if ((long long)tt * pr.H * pr.W >= (1LL << 30)) return BSA_ERR_UNSUPPORTED;
+    x.slab = tt * pr.H * pr.W;
     if (x.nb > kMaxBlocks) return BSA_ERR_UNSUPPORTED;
     *g = x;
     return BSA_OK;
@@ -81,10 +82,26 @@ int drift_chunks(const Geom& g) {
 
 int text_splits(const Geom& g) { return (g.nb + attn::kTextChunk - 1) / attn::kTextChunk; }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Attention workspace: [perm: nb*B int32][text partial O: items*BQ*d fp32][text lse: items*BQ fp32]
+size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(int)); }
+
 size_t attention_ws_bytes(const Geom& g) {
-    if (g.nbt == 0) return 0;
-    const size_t items = (size_t)g.heads * g.nbt * text_splits(g);
-    return items * attn::BQ * (size_t)(g.d + 1) * sizeof(float);
+    size_t bytes = perm_bytes(g);
+    if (g.nbt > 0) {
+        const size_t items = (size_t)g.heads * g.nbt * text_splits(g);
+        bytes += align256(items * attn::BQ * (size_t)g.d * sizeof(float));
+        bytes += align256(items * attn::BQ * sizeof(float));
+    }
+    return bytes;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return n;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
@@ -92,14 +109,21 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA
 int launch_status() { return cuda_status(cudaGetLastError()); }
 
 template <int D, int BK>
-int launch_attention(const attn::Params& P, int items, cudaStream_t st) {
+int launch_attention(const attn::Params& P, cudaStream_t st) {
     using C = attn::Cfg<D, BK>;
     // set on every call: the attribute is per device and the call is cheap
     if (cudaFuncSetAttribute(attn::sparse_attention_kernel<D, BK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return BSA_ERR_CUDA;
-    attn::sparse_attention_kernel<D, BK><<<items, attn::kThreads, C::SMEM, st>>>(P);
+    const int sms = sm_count();
+    if (sms <= 0) return BSA_ERR_CUDA;
+    const int grid = P.n_items < sms ? P.n_items : sms;   // persistent: one CTA per SM
+    const int total = P.g.nb * P.g.B;
+    attn::perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(P.g, const_cast<int*>(P.perm));
     int rc = launch_status();
+    if (rc != BSA_OK) return rc;
+    attn::sparse_attention_kernel<D, BK><<<grid, attn::kThreads, C::SMEM, st>>>(P);
+    rc = launch_status();
     if (rc != BSA_OK) return rc;
     if (P.n_text_items > 0) {
         dim3 grid(P.g.heads * P.g.nbt, attn::BQ);
@@ -242,8 +266,8 @@ int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(cnt) || !aligned16(O))
         return BSA_ERR_ALIGN;
     const size_t need = attention_ws_bytes(g);
-    if (need > 0 && (ws == nullptr || ws_bytes < need)) return BSA_ERR_WORKSPACE;
-    if (need > 0 && !aligned16(ws)) return BSA_ERR_ALIGN;
+    if (ws == nullptr || ws_bytes < need) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
     attn::Params P;
     P.g = g;
     P.Q = Q;
@@ -254,15 +278,19 @@ int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     P.O = O;
     P.nsplit = g.nbt > 0 ? text_splits(g) : 1;
     P.n_text_items = g.heads * g.nbt * (g.nbt > 0 ? P.nsplit : 0);
-    P.part_o = need > 0 ? static_cast<float*>(ws) : nullptr;
-    P.part_lse = need > 0 ? P.part_o + (size_t)P.n_text_items * attn::BQ * g.d : nullptr;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    P.perm = reinterpret_cast<int*>(w);
+    P.part_o = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g)) : nullptr;
+    P.part_lse = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g) +
+                                                      align256((size_t)P.n_text_items * attn::BQ * g.d * sizeof(float)))
+                           : nullptr;
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
-    const int items = P.n_text_items + g.heads * g.nbv;
+    P.n_items = P.n_text_items + g.heads * g.nbv;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (g.d == 128 && g.B == 128) return launch_attention<128, 128>(P, items, st);
-    if (g.d == 128) return launch_attention<128, 64>(P, items, st);
-    if (g.B == 128) return launch_attention<64, 128>(P, items, st);
-    return launch_attention<64, 64>(P, items, st);
+    if (g.d == 128 && g.B == 128) return launch_attention<128, 128>(P, st);
+    if (g.d == 128) return launch_attention<128, 64>(P, st);
+    if (g.B == 128) return launch_attention<64, 128>(P, st);
+    return launch_attention<64, 64>(P, st);
 }
 
 int bsa_device_status(bsa_stream_t stream) {

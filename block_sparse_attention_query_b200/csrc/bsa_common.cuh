@@ -20,7 +20,7 @@ struct Geom {
     int tt, th, tw;       // tile shape
     int nb, nbv, nbt;     // blocks: total, video, text
     int Nv;               // video tokens
-    long long slab;       // tokens per full tile slab along t: tt*H*W
+    int slab;             // tokens per full tile slab along t: tt*H*W
 };
 
 // Raster token index held by block slot `s` (0 <= s < nb*B), or -1 for a padding slot.
@@ -33,8 +33,8 @@ __host__ __device__ inline int slot_to_token(const Geom& g, int s) {
         return t < g.text ? g.Nv + t : -1;
     }
     if (s >= g.Nv) return -1;
-    const int a = (int)(s / g.slab);                       // tile slab along t
-    int r = (int)(s - (long long)a * g.slab);
+    const int a = s / g.slab;                              // tile slab along t
+    int r = s - a * g.slab;
     const int ta = min(g.tt, g.T - a * g.tt);              // frames in this slab
     const int row_tokens = ta * g.th * g.W;                 // tokens per full tile row
     const int b = r / row_tokens;
@@ -100,13 +100,15 @@ __device__ inline void mbar_arrive(uint64_t* bar) {
                  ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Suspends the thread (no spinning) until the phase with the given parity completes or the
+// hinted time (in ns) passes; returns whether it completed.
 __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u) : "memory");
     return ok != 0;
 }
 
@@ -115,12 +117,9 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    uint32_t spins = 0;
     while (!mbar_try_wait(bar, parity)) {
-        if ((++spins & 63u) == 0) {
-            if (error_raised()) return false;
-            if (clock64() - t0 > kWaitLimitCycles) { raise_error(BSA_ERR_TIMEOUT); return false; }
-        }
+        if (error_raised()) return false;
+        if (clock64() - t0 > kWaitLimitCycles) { raise_error(BSA_ERR_TIMEOUT); return false; }
     }
     return true;
 }

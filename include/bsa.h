@@ -154,8 +154,9 @@ int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* 
  *              indices in [0, nb) are accepted; a bad entry sets BSA_ERR_DEVICE_ARG in the
  *              device error word and the row's output is unspecified).
  *   O          [heads, tokens, d] bf16 out, raster order. Every real token is written.
- *   ws         at least plan.attention_workspace_bytes (partial results of the dense text
- *              rows, which are split across CTAs). */
+ *   ws         at least plan.attention_workspace_bytes, always required: the block-slot ->
+ *              token table, and the partial results of the dense text rows, which are split
+ *              across CTAs and merged. */
 int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                          const bsa_bf16* V, const int* idx, const int* cnt, bsa_bf16* O,
                          void* ws, size_t ws_bytes, bsa_stream_t stream);

@@ -99,8 +99,9 @@ def test_calls_reject_bad_pointers_before_launch():
     assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(float("nan")), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
     assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(0.05), 0, a, a, a, 8, None) == bsa.BSA_ERR_WORKSPACE
     assert L.bsa_drift_check(pr, a, a, a, None, ctypes.c_float(0.05), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
-    assert L.bsa_sparse_attention(pr, a, a, a, a, a, None, a, 0, None) == bsa.BSA_ERR_ARG
-    assert L.bsa_sparse_attention(pr, a, a, mis, a, a, a, a, 0, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_sparse_attention(pr, a, a, a, a, a, None, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_sparse_attention(pr, a, a, mis, a, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_sparse_attention(pr, a, a, a, a, a, a, None, 1 << 20, None) == bsa.BSA_ERR_WORKSPACE
     text = bsa.problem(2, 64, 4, 16, 16, 64, 64)
     need = bsa.bsa_plan(text).attention_workspace_bytes
     assert need > 0
