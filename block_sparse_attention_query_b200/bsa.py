@@ -20,6 +20,7 @@ BSA_ERR_WORKSPACE = -4
 BSA_ERR_CUDA = -5
 BSA_ERR_TIMEOUT = -6
 BSA_ERR_DEVICE_ARG = -7
+BSA_ERR_SCRATCH_LIMIT = -8
 
 BSA_SCORE_MEANPOOL = 0
 BSA_SCORE_PARK = 1
@@ -62,6 +63,9 @@ EXPORTS = {
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p]),
+    "bsa_drift_check_noalloc": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "bsa_sparse_attention": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
@@ -147,6 +151,13 @@ def bsa_drift_check(prob, Q, K, Q_ref, K_ref, tau, force_all, drift, refresh, ws
                               ctypes.c_float(tau), int(force_all), _ptr(drift), _ptr(refresh), _ptr(ws),
                               ws.numel() * ws.element_size() if ws is not None else 0,
                               _stream(stream)), "bsa_drift_check")
+
+
+def bsa_drift_check_noalloc(prob, Q, K, Q_ref, K_ref, tau, force_all, drift, refresh, stream=None):
+    """bsa_drift_check with the library's static scratch instead of a caller workspace."""
+    check(lib.bsa_drift_check_noalloc(ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(Q_ref), _ptr(K_ref),
+                                      ctypes.c_float(tau), int(force_all), _ptr(drift), _ptr(refresh),
+                                      _stream(stream)), "bsa_drift_check_noalloc")
 
 
 def bsa_sparse_attention(prob, Q, K, V, idx, cnt, O, ws, stream=None):

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "bsa_common.cuh"
 #include "score.cuh"
@@ -293,6 +294,65 @@ int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     return launch_attention<64, 64>(P, st);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Drift check without a caller workspace.
+//
+// Some callers cannot allocate device memory when they call in: inference servers and
+// real-time pipelines that reserve all device memory at start-up and forbid allocation
+// afterwards, and plugin interfaces that hand a kernel only its input and output buffers
+// with no way to ask for scratch space. bsa_drift_check_noalloc serves them: its float64
+// partial sums live in the library's own static device array below instead of a caller
+// workspace. That array exists once per device that loads the library and stays until the
+// process exits; every call on a device shares it.
+namespace {
+
+constexpr size_t kNoallocDriftDoubles = 262144;   // 2 MiB: heads * chunks * 4 doubles
+static __device__ __align__(256) double g_noalloc_drift_scratch[kNoallocDriftDoubles];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+double* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the static scratch on the current device, looked up once per device.
+// The name g_noalloc_drift_scratch is only a host-side stand-in; kernels must get this
+// address instead.
+int noalloc_scratch(double** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_drift_scratch) != cudaSuccess) return BSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<double*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return BSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                            bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all, float* drift,
+                            int* refresh, bsa_stream_t stream) {
+    Geom g;
+    const int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    const size_t need = (size_t)g.heads * drift_chunks(g) * 4;
+    if (need > kNoallocDriftDoubles) return BSA_ERR_SCRATCH_LIMIT;
+    double* scratch = nullptr;
+    const int sc = noalloc_scratch(&scratch);
+    if (sc != BSA_OK) return sc;
+    // every partial that the finalize pass reads is written first by the partial pass of
+    // the same call, so the shared array needs no clearing between calls
+    return bsa_drift_check(prob, Q, K, Q_ref, K_ref, tau, force_all, drift, refresh, scratch,
+                           kNoallocDriftDoubles * sizeof(double), stream);
+}
+
 int bsa_device_status(bsa_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
@@ -315,6 +375,9 @@ const char* bsa_error_string(int status) {
         case BSA_ERR_CUDA: return "CUDA launch or runtime error";
         case BSA_ERR_TIMEOUT: return "device: a bounded wait in a kernel ran out";
         case BSA_ERR_DEVICE_ARG: return "device: kept-block index or count out of range";
+        case BSA_ERR_SCRATCH_LIMIT:
+            return "problem too large for the static scratch of bsa_drift_check_noalloc "
+                   "(needs heads * ceil(tokens * d / 16384) <= 65536)";
         default: return "unknown status";
     }
 }

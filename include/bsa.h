@@ -59,6 +59,7 @@ typedef struct CUstream_st* bsa_stream_t;  /* identical to cudaStream_t */
 #define BSA_ERR_CUDA        -5   /* a CUDA launch or runtime call failed */
 #define BSA_ERR_TIMEOUT     -6   /* device: a bounded wait inside a kernel ran out */
 #define BSA_ERR_DEVICE_ARG  -7   /* device: a kept-block index or count was out of range */
+#define BSA_ERR_SCRATCH_LIMIT -8 /* problem exceeds the static scratch of bsa_drift_check_noalloc */
 
 /* scorers (PARK, Abstract) */
 #define BSA_SCORE_MEANPOOL   0   /* softmax_j( mean(Q in block i) . mean(K in block j) / sqrt(d) ) */
@@ -143,6 +144,23 @@ int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* 
                     bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all,
                     float* drift, int* refresh,
                     void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* bsa_drift_check for callers that cannot allocate device memory. The paper has no
+ * counterpart; this is a deployment convenience. Some callers cannot call cudaMalloc when
+ * they call in: servers and real-time pipelines that reserve all device memory at start-up
+ * and forbid allocation afterwards, and plugin interfaces that pass a kernel only its inputs
+ * and outputs. This entry point takes no workspace and allocates nothing: its scratch is a
+ * 2 MiB static device array inside the library (held on every device that loads the library
+ * until the process exits).
+ *   Arguments, results and determinism are those of bsa_drift_check.
+ *   Limit: heads * ceil(tokens * d / 16384) <= 65536; larger problems return
+ *          BSA_ERR_SCRATCH_LIMIT and launch nothing.
+ *   The first call on a device looks up the scratch address on that device (make that first
+ *   call before any stream capture). All calls on a device share the one array: calls that
+ *   may overlap on the GPU (different streams without ordering) race and must not be made. */
+int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                            bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all,
+                            float* drift, int* refresh, bsa_stream_t stream);
 
 /* Block-sparse attention (PARK, Abstract: attention computed only within the retrieved
  * blocks). For every real query t of query block i of head h:
