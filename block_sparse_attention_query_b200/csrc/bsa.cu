@@ -190,8 +190,11 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     const float scale = 1.0f / std::sqrt((float)g.d);
     if (prob->score_mode == BSA_SCORE_MEANPOOL) {
         const int nbp = (g.nb + 3) & ~3;
-        const bool wide = g.nb > 1024;
-        const int R = wide ? 16 : 32;
+        // rows per CTA: as many as keep >= 2 CTAs per SM busy (fewer rows = more CTAs, but
+        // each CTA re-reads every pooled key of its head from L2); 16 at most past 1024 blocks
+        int R = 32;
+        if (g.nb > 1024) R = 16;
+        while (R > 8 && (long long)((g.nb + R - 1) / R) * g.heads < 296) R >>= 1;
         const size_t smem = (size_t)(R * g.d + R * nbp) * sizeof(float);
         const dim3 grid((g.nb + R - 1) / R, g.heads);
 #define BSA_MP(DD, RR)                                                                             \
@@ -201,8 +204,8 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
             return BSA_ERR_CUDA;                                                                   \
         meanpool_score_kernel<DD, RR><<<grid, 256, smem, st>>>(g, qbar, kbar, head_mask, scores, scale); \
     } while (0)
-        if (g.d == 128) { if (wide) BSA_MP(128, 16); else BSA_MP(128, 32); }
-        else { if (wide) BSA_MP(64, 16); else BSA_MP(64, 32); }
+        if (g.d == 128) { if (R == 32) BSA_MP(128, 32); else if (R == 16) BSA_MP(128, 16); else BSA_MP(128, 8); }
+        else { if (R == 32) BSA_MP(64, 32); else if (R == 16) BSA_MP(64, 16); else BSA_MP(64, 8); }
 #undef BSA_MP
         return launch_status();
     }
