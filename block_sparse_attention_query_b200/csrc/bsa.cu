@@ -220,13 +220,29 @@ int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p
     if (scores == nullptr || p == nullptr || idx == nullptr || cnt == nullptr) return BSA_ERR_ARG;
     if (!aligned16(scores) || !aligned16(idx) || !aligned16(cnt) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // pass 1: one warp per video row extracts the top-p prefix (rows of up to 1024 blocks)
+    const int sort_all = (g.nb > 1024 || g.nbt > 64) ? 1 : 0;
+    if (!sort_all) {
+        const long long rows = (long long)g.heads * g.nb;
+        const int wgrid = (int)((rows + 7) / 8);
+#define BSA_WSEL(EE) select_topp_warp_kernel<EE><<<wgrid, 256, 0, st>>>(g, scores, p, head_mask, idx, cnt)
+        if (g.nb <= 64) BSA_WSEL(2);
+        else if (g.nb <= 128) BSA_WSEL(4);
+        else if (g.nb <= 256) BSA_WSEL(8);
+        else if (g.nb <= 512) BSA_WSEL(16);
+        else BSA_WSEL(32);
+#undef BSA_WSEL
+        const int rc = launch_status();
+        if (rc != BSA_OK) return rc;
+    }
+    // pass 2: one CTA per remaining row (text rows, p >= 1, overflow, or all) sorts it fully
     const dim3 grid(g.nb, g.heads);
-    if (g.nb <= 64) select_topp_kernel<64><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
-    else if (g.nb <= 128) select_topp_kernel<128><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
-    else if (g.nb <= 256) select_topp_kernel<256><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
-    else if (g.nb <= 512) select_topp_kernel<512><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
-    else if (g.nb <= 1024) select_topp_kernel<1024><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
-    else select_topp_kernel<2048><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt);
+    if (g.nb <= 64) select_topp_kernel<64><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
+    else if (g.nb <= 128) select_topp_kernel<128><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
+    else if (g.nb <= 256) select_topp_kernel<256><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
+    else if (g.nb <= 512) select_topp_kernel<512><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
+    else if (g.nb <= 1024) select_topp_kernel<1024><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
+    else select_topp_kernel<2048><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
     return launch_status();
 }
 

@@ -15,11 +15,15 @@
 namespace bsa {
 
 constexpr int kSelectThreads = 256;
+constexpr int kWarpSelectCap = 64;      // extractions before a row falls back to the full sort
 
+// Rows the per-warp kernel below does not finish: text query rows and heads with p >= 1
+// (every block kept), rows it marked with cnt = -1 (more than kWarpSelectCap blocks to
+// extract), and every row when sort_all is set (more than 1024 blocks per row).
 template <int N2>
 __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
     Geom g, const float* __restrict__ scores, const float* __restrict__ p,
-    const int* __restrict__ head_mask, int* __restrict__ idx, int* __restrict__ cnt) {
+    const int* __restrict__ head_mask, int* __restrict__ idx, int* __restrict__ cnt, int sort_all) {
     constexpr int NT = kSelectThreads;
     constexpr int E = (N2 + NT - 1) / NT;   // sorted elements owned per thread in the scan
     __shared__ unsigned long long key[N2];
@@ -30,6 +34,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
     const int i = blockIdx.x, h = blockIdx.y;
     if (head_mask != nullptr && head_mask[h] == 0) return;
     const int nb = g.nb;
+    if (!sort_all && i < g.nbv && p[h] < 1.0f && cnt[(size_t)h * nb + i] != -1) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float* row = scores + ((size_t)h * nb + i) * nb;
 
@@ -129,6 +134,113 @@ __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
         if (flags[e]) out[base++] = (int)(uint32_t)key[tid * E + e];
     }
     if (tid == 0) cnt[(size_t)h * nb + i] = total;
+}
+
+
+// One warp per video query row with p < 1 (rows up to 1024 blocks). Lane l holds the keys
+// of blocks l, l+32, ...: key = ~float_bits(score), so an ascending key order is score
+// descending, and among equal keys the lower block index wins. The warp extracts the best
+// remaining block, adds its score to a float32 running sum (sequentially, in sorted order)
+// and stops once the sum reaches p -- usually after a handful of blocks. The kept list is
+// then merged with the forced text key blocks in the same order. A row that needs more than
+// kWarpSelectCap extractions is marked cnt = -1 for the sorting kernel.
+template <int E>
+__global__ void __launch_bounds__(256) select_topp_warp_kernel(
+    Geom g, const float* __restrict__ scores, const float* __restrict__ p,
+    const int* __restrict__ head_mask, int* __restrict__ idx, int* __restrict__ cnt) {
+    __shared__ int kept_s[8][kWarpSelectCap];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = g.nb;
+    const long long row = (long long)blockIdx.x * 8 + warp;
+    if (row >= (long long)g.heads * nb) return;
+    const int h = (int)(row / nb), i = (int)(row - (long long)h * nb);
+    if (i >= g.nbv) return;                                   // text rows: sorting kernel
+    if (head_mask != nullptr && head_mask[h] == 0) return;
+    const float pth = p[h];
+    if (!(pth < 1.0f)) return;                                // keep-all rows: sorting kernel
+    const float* srow = scores + (size_t)row * nb;
+    uint32_t key[E];
+#pragma unroll
+    for (int m = 0; m < E; ++m) {
+        const int j = lane + 32 * m;
+        uint32_t k = 0xFFFFFFFFu;
+        if (j < nb) {
+            const float sc = srow[j];
+            k = ~((sc > 0.f) ? __float_as_uint(sc) : 0u);    // not > 0 (0, -0, NaN) orders as 0
+        }
+        key[m] = k;
+    }
+    // lane-local best untaken block as (key << 32 | index); all ones when none is left (no
+    // real block has that value: indices stay below 2^31)
+    uint32_t taken = 0;                                     // bit m: block lane + 32m retired
+#pragma unroll
+    for (int m = 0; m < E; ++m)
+        if (lane + 32 * m >= nb) taken |= 1u << m;
+    auto local_best = [&]() -> unsigned long long {
+        unsigned long long b = ~0ull;
+#pragma unroll
+        for (int m = 0; m < E; ++m) {
+            const unsigned long long c = ((unsigned long long)key[m] << 32) | (uint32_t)(lane + 32 * m);
+            if (!((taken >> m) & 1u) && c < b) b = c;
+        }
+        return b;
+    };
+    unsigned long long mine = local_best();
+    float cum = 0.f;
+    int n = 0;
+    bool done = false;
+    while (!done && n < kWarpSelectCap) {
+        unsigned long long best = mine;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other < best ? other : best;
+        }
+        if (best == ~0ull) { done = true; break; }            // every block kept: sum stayed < p
+        const uint32_t bkey = (uint32_t)(best >> 32);
+        const int bj = (int)(uint32_t)best;
+        if (lane == 0) kept_s[warp][n] = bj;
+        ++n;
+        cum += __uint_as_float(~bkey);                       // sequential float32 sum
+        if (cum >= pth) done = true;
+        if ((bj & 31) == lane) {                             // owner retires the block
+            taken |= 1u << (bj >> 5);
+            mine = local_best();
+        }
+    }
+    if (!done) {                                            // too many blocks: full sort
+        if (lane == 0) cnt[row] = -1;
+        return;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        // merge the kept prefix (already in key order) with the forced text blocks, taken
+        // in key order too (at most 64 text blocks reach this kernel)
+        auto key_of = [&](int j) -> unsigned long long {
+            const float sc = srow[j];
+            return ((unsigned long long)(~((sc > 0.f) ? __float_as_uint(sc) : 0u)) << 32) | (uint32_t)j;
+        };
+        int* out = idx + (size_t)row * nb;
+        unsigned long long used = 0;                     // bit t - nbv: text block placed
+        for (int q = 0; q < n; ++q)
+            if (kept_s[warp][q] >= g.nbv) used |= 1ull << (kept_s[warp][q] - g.nbv);
+        int a = 0, o = 0;
+        while (true) {
+            int bt = -1;
+            unsigned long long bk = ~0ull;
+            for (int t = g.nbv; t < nb; ++t) {
+                if ((used >> (t - g.nbv)) & 1ull) continue;
+                const unsigned long long k = key_of(t);
+                if (k < bk) { bk = k; bt = t; }
+            }
+            if (bt < 0) break;
+            used |= 1ull << (bt - g.nbv);
+            while (a < n && key_of(kept_s[warp][a]) < bk) out[o++] = kept_s[warp][a++];
+            out[o++] = bt;
+        }
+        while (a < n) out[o++] = kept_s[warp][a++];
+        cnt[row] = o;
+    }
 }
 
 }  // namespace bsa

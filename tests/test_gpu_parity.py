@@ -353,3 +353,25 @@ def test_full_size_masks_and_sampled_attention(name, mode):
     # combination of V rows (bounded by the V range)
     vmax = float(np.abs(O.bf16_to_f64(c.Vb)).max())
     assert torch.isfinite(got).all() and float(got.abs().max()) <= vmax + 1e-2
+
+
+@pytest.mark.parametrize("conc,p", [(50.0, 0.95), (0.3, 0.9), (5.0, 0.999)])
+def test_select_flat_and_peaked_rows(conc, p):
+    # flat rows need far more than the per-warp extraction cap and fall back to the full
+    # sort; peaked rows stop early. Both must match the oracle's selection on the same
+    # float32 scores (only the 1e-5 cumulative-mass window may differ).
+    bsa = _bsa()
+    L = O.block_layout(4, 64, 64, 0, 64)          # 256 blocks, no text
+    heads = 3
+    rng = np.random.default_rng(int(conc * 10) + int(p * 1000))
+    S = rng.dirichlet(np.full(L.nb, conc), size=(heads, L.nb)).astype(np.float32)
+    prob = bsa.problem(heads, 64, 4, 64, 64, 0, 64)
+    pd = torch.full((heads,), p, dtype=torch.float32, device="cuda")
+    idx = torch.full((heads, L.nb, L.nb), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(heads, L.nb, dtype=torch.int32, device="cuda")
+    bsa.bsa_select_topp(prob, torch.from_numpy(S).cuda(), pd, None, idx, cnt)
+    _status_ok()
+    res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, np.full(heads, p), L)
+    assert res["mismatch"] == 0 and res["tie"] == 0, res
+    if conc >= 5.0:
+        assert cnt.cpu().numpy().mean() > 64       # the fallback path was exercised
