@@ -695,11 +695,5 @@ __global__ void merge_text_kernel(Params P) {
     P.O[(size_t)h * g.N * D + (size_t)tok * D + threadIdx.x] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
 }
 
-// perm[s] = raster token of block slot s (-1 = padding), for s in [0, nb*B).
-__global__ void perm_kernel(Geom g, int* perm) {
-    const int s = blockIdx.x * blockDim.x + threadIdx.x;
-    if (s < g.nb * g.B) perm[s] = slot_to_token(g, s);
-}
-
 }  // namespace attn
 }  // namespace bsa

@@ -74,7 +74,13 @@ int make_geom(const bsa_problem* prob, Geom* g) {
     return BSA_OK;
 }
 
-size_t pooled_bytes(const Geom& g) { return (size_t)2 * g.heads * g.nb * g.d * sizeof(float); }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(int)); }
+
+// Score workspace: [pooled Q means | pooled K means: heads*nb*d fp32 each][block-slot table]
+size_t pooled_bytes(const Geom& g) { return align256((size_t)2 * g.heads * g.nb * g.d * sizeof(float)); }
+size_t score_ws_bytes(const Geom& g) { return pooled_bytes(g) + perm_bytes(g); }
 
 int drift_chunks(const Geom& g) {
     const long long elems = (long long)g.N * g.d;
@@ -83,10 +89,7 @@ int drift_chunks(const Geom& g) {
 
 int text_splits(const Geom& g) { return (g.nb + attn::kTextChunk - 1) / attn::kTextChunk; }
 
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
 // Attention workspace: [perm: nb*B int32][text partial O: items*BQ*d fp32][text lse: items*BQ fp32]
-size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(int)); }
 
 size_t attention_ws_bytes(const Geom& g) {
     size_t bytes = perm_bytes(g);
@@ -120,7 +123,7 @@ int launch_attention(const attn::Params& P, cudaStream_t st) {
     if (sms <= 0) return BSA_ERR_CUDA;
     const int grid = P.n_items < sms ? P.n_items : sms;   // persistent: one CTA per SM
     const int total = P.g.nb * P.g.B;
-    attn::perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(P.g, const_cast<int*>(P.perm));
+    perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(P.g, const_cast<int*>(P.perm));
     int rc = launch_status();
     if (rc != BSA_OK) return rc;
     attn::sparse_attention_kernel<D, BK><<<grid, attn::kThreads, C::SMEM, st>>>(P);
@@ -152,7 +155,7 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.tile_t = g.tt;
     info.tile_h = g.th;
     info.tile_w = g.tw;
-    info.score_workspace_bytes = pooled_bytes(g);
+    info.score_workspace_bytes = score_ws_bytes(g);
     info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
     info.attention_workspace_bytes = attention_ws_bytes(g);
     *out = info;
@@ -176,16 +179,20 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || scores == nullptr) return BSA_ERR_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
-    if (ws == nullptr || ws_bytes < pooled_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (ws == nullptr || ws_bytes < score_ws_bytes(g)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* qbar = static_cast<float*>(ws);
     float* kbar = qbar + (size_t)g.heads * g.nb * g.d;
+    int* perm = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pooled_bytes(g));
+    const int total = g.nb * g.B;
+    perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(g, perm);
+    if ((rc = launch_status()) != BSA_OK) return rc;
     const dim3 pgrid(g.nb, g.heads);
-    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
-    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
-    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
-    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, head_mask, qbar, kbar);
+    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
+    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
+    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
+    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
     if ((rc = launch_status()) != BSA_OK) return rc;
     const float scale = 1.0f / std::sqrt((float)g.d);
     if (prob->score_mode == BSA_SCORE_MEANPOOL) {
@@ -195,7 +202,7 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
         int R = 32;
         if (g.nb > 1024) R = 16;
         while (R > 8 && (long long)((g.nb + R - 1) / R) * g.heads < 296) R >>= 1;
-        const size_t smem = (size_t)(R * g.d + R * nbp) * sizeof(float);
+        const size_t smem = (size_t)(R * g.d + kScoreKeyChunk * (g.d + 4) + R * nbp) * sizeof(float);
         const dim3 grid((g.nb + R - 1) / R, g.heads);
 #define BSA_MP(DD, RR)                                                                             \
     do {                                                                                           \

@@ -51,6 +51,13 @@ __host__ __device__ inline int slot_to_token(const Geom& g, int s) {
     return ((a * g.tt + lt) * g.H + (b * g.th + ly)) * g.W + (c * g.tw + lx);
 }
 
+// Block-slot table: perm[s] = raster token of block slot s (-1 = padding), s < nb*B.
+// Built once per call, so kernels look tokens up instead of dividing per row.
+__global__ void perm_kernel(Geom g, int* perm) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s < g.nb * g.B) perm[s] = slot_to_token(g, s);
+}
+
 // Number of real tokens in block i.
 __host__ __device__ inline int block_count(const Geom& g, int i) {
     if (i < g.nbv) return min(g.B, g.Nv - i * g.B);

@@ -29,6 +29,7 @@ __device__ inline void accum_bf16x8(float (&acc)[8], const uint4& v) {
 template <int D, int B>
 __global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __restrict__ Q,
                                                    const bsa_bf16* __restrict__ K,
+                                                   const int* __restrict__ perm,
                                                    const int* __restrict__ head_mask,
                                                    float* __restrict__ qbar, float* __restrict__ kbar) {
     constexpr int CH = D / 8;               // 16-byte chunks per row
@@ -41,7 +42,7 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __res
 
     int tok[NIT];
 #pragma unroll
-    for (int k = 0; k < NIT; ++k) tok[k] = slot_to_token(g, i * B + rs + k * RPP);
+    for (int k = 0; k < NIT; ++k) tok[k] = __ldg(perm + i * B + rs + k * RPP);
     uint4 vq[NIT], vk[NIT];
 #pragma unroll
     for (int k = 0; k < NIT; ++k) {
@@ -78,55 +79,63 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __res
     }
 }
 
-// grid (ceil(nb/R), heads), 256 threads; dynamic smem = (R*D + R*nbp) floats.
-// Rows i0..i0+R-1 of head h: logits against every key block, then row softmax.
+// grid (ceil(nb/R), heads), 256 threads; dynamic smem = (R*D + KC*(D+4) + R*nbp) floats.
+// Rows i0..i0+R-1 of head h: logits against every key block (pooled keys staged through
+// shared memory KC at a time), then row softmax.
+constexpr int kScoreKeyChunk = 64;
+
 template <int D, int R>
 __global__ void __launch_bounds__(256) meanpool_score_kernel(Geom g, const float* __restrict__ qbar,
                                                              const float* __restrict__ kbar,
                                                              const int* __restrict__ head_mask,
                                                              float* __restrict__ scores, float scale) {
+    constexpr int KC = kScoreKeyChunk;
+    constexpr int KS = D + 4;              // padded row stride of the staged keys
+    constexpr int RPT = R / 4;             // rows per thread (4 row groups x 64 keys)
     extern __shared__ float4 smem_f4[];
     const int h = blockIdx.y, i0 = blockIdx.x * R;
     if (head_mask != nullptr && head_mask[h] == 0) return;
     const int nb = g.nb;
     const int nbp = (nb + 3) & ~3;
     float* sq = reinterpret_cast<float*>(smem_f4);      // [R][D]
-    float* slog = sq + R * D;                            // [R][nbp]
+    float* sk = sq + R * D;                              // [KC][KS]
+    float* slog = sk + KC * KS;                          // [R][nbp]
     const float* qh = qbar + (size_t)h * nb * D;
     const float* kh = kbar + (size_t)h * nb * D;
     for (int e = threadIdx.x; e < R * D; e += 256) {
         const int r = e / D;
         sq[e] = (i0 + r < nb) ? qh[(size_t)(i0 + r) * D + (e % D)] : 0.f;
     }
-    __syncthreads();
+    const int kk = threadIdx.x % KC, rg = threadIdx.x / KC;   // key in chunk, row group
     const float4* sq4 = reinterpret_cast<const float4*>(sq);
-    for (int jb = 0; jb < nb; jb += 512) {
-        const int ja = jb + threadIdx.x, jbb = ja + 256;
-        const float4* ka = reinterpret_cast<const float4*>(kh + (size_t)min(ja, nb - 1) * D);
-        const float4* kb = reinterpret_cast<const float4*>(kh + (size_t)min(jbb, nb - 1) * D);
-        float acc0[R], acc1[R];
+    for (int j0 = 0; j0 < nb; j0 += KC) {
+        __syncthreads();                                 // previous chunk consumed
+        for (int e = threadIdx.x; e < KC * (D / 4); e += 256) {
+            const int j = e / (D / 4), c4 = e % (D / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kh + (size_t)(j0 + j) * D) + c4);
+            *reinterpret_cast<float4*>(sk + j * KS + c4 * 4) = v;
+        }
+        __syncthreads();
+        float acc[RPT];
 #pragma unroll
-        for (int r = 0; r < R; ++r) { acc0[r] = 0.f; acc1[r] = 0.f; }
-#pragma unroll 2
+        for (int q = 0; q < RPT; ++q) acc[q] = 0.f;
+        const float4* krow = reinterpret_cast<const float4*>(sk + kk * KS);
+#pragma unroll 4
         for (int c4 = 0; c4 < D / 4; ++c4) {
-            const float4 a = __ldg(ka + c4), b = __ldg(kb + c4);
+            const float4 kv = krow[c4];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float4 q = sq4[r * (D / 4) + c4];
-                acc0[r] = fmaf(q.x, a.x, acc0[r]);
-                acc0[r] = fmaf(q.y, a.y, acc0[r]);
-                acc0[r] = fmaf(q.z, a.z, acc0[r]);
-                acc0[r] = fmaf(q.w, a.w, acc0[r]);
-                acc1[r] = fmaf(q.x, b.x, acc1[r]);
-                acc1[r] = fmaf(q.y, b.y, acc1[r]);
-                acc1[r] = fmaf(q.z, b.z, acc1[r]);
-                acc1[r] = fmaf(q.w, b.w, acc1[r]);
+            for (int q = 0; q < RPT; ++q) {
+                const float4 qv = sq4[(rg * RPT + q) * (D / 4) + c4];
+                acc[q] = fmaf(qv.x, kv.x, acc[q]);
+                acc[q] = fmaf(qv.y, kv.y, acc[q]);
+                acc[q] = fmaf(qv.z, kv.z, acc[q]);
+                acc[q] = fmaf(qv.w, kv.w, acc[q]);
             }
         }
+        if (j0 + kk < nb) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            if (ja < nb) slog[r * nbp + ja] = acc0[r] * scale;
-            if (jbb < nb) slog[r * nbp + jbb] = acc1[r] * scale;
+            for (int q = 0; q < RPT; ++q) slog[(rg * RPT + q) * nbp + j0 + kk] = acc[q] * scale;
         }
     }
     __syncthreads();
