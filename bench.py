@@ -252,8 +252,10 @@ def run_ours(args, ws, rank, local):
         e2e = {"value": round(e2e_ms / ws, 4), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
 
-    # drift (2) + pool, score (2) + select (1) + block-slot table, attention (2) [+ text merge]
-    launches_per_step = 2 + 2 + 1 + 2 + (1 if plan.nb_text > 0 else 0)
+    # drift (2) + block-slot table, pool, score (3) + select (warp pass unless every row is
+    # sorted, sort pass) + block-slot table, attention (2) [+ text merge]
+    sort_all = plan.nb > 1024 or plan.nb_text > 64
+    launches_per_step = 2 + 3 + (1 if sort_all else 2) + 2 + (1 if plan.nb_text > 0 else 0)
     value = ms_step / ws
     line = {
         "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": ws,

@@ -242,8 +242,10 @@ int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p
         const int rc = launch_status();
         if (rc != BSA_OK) return rc;
     }
-    // pass 2: one CTA per remaining row (text rows, p >= 1, overflow, or all) sorts it fully
-    const dim3 grid(g.nb, g.heads);
+    // pass 2: CTAs walk the rows (grid-stride) and fully sort the remaining ones (text rows,
+    // p >= 1, overflow, or all of them)
+    const int rows_all = g.heads * g.nb;
+    const int grid = sort_all ? rows_all : (rows_all < 1184 ? rows_all : 1184);
     if (g.nb <= 64) select_topp_kernel<64><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
     else if (g.nb <= 128) select_topp_kernel<128><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
     else if (g.nb <= 256) select_topp_kernel<256><<<grid, kSelectThreads, 0, st>>>(g, scores, p, head_mask, idx, cnt, sort_all);
@@ -277,8 +279,10 @@ int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* 
     drift_partial_kernel<<<grid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, part);
     int r2 = launch_status();
     if (r2 != BSA_OK) return r2;
-    drift_finalize_kernel<<<grid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, tau,
-                                                         part, drift, refresh);
+    // with force_all the snapshot was taken in the first pass: one CTA per head publishes
+    const dim3 fgrid(force_all ? 1 : chunks, g.heads);
+    drift_finalize_kernel<<<fgrid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, tau,
+                                                          part, drift, refresh, chunks);
     return launch_status();
 }
 

@@ -102,11 +102,12 @@ __device__ inline double rel_change(double diff2, double ref2) {
     return sqrt(diff2 / ref2);
 }
 
+// grid (chunks or 1, heads): nchunks is the number of partials per head.
 __global__ void __launch_bounds__(kDriftThreads) drift_finalize_kernel(
     const bsa_bf16* __restrict__ Q, const bsa_bf16* __restrict__ K, bsa_bf16* Qref,
     bsa_bf16* Kref, long long elems, int force_all, float tau,
-    const double* __restrict__ part, float* __restrict__ drift, int* __restrict__ refresh) {
-    const int c = blockIdx.x, h = blockIdx.y, nchunks = gridDim.x;
+    const double* __restrict__ part, float* __restrict__ drift, int* __restrict__ refresh, int nchunks) {
+    const int c = blockIdx.x, h = blockIdx.y;
     __shared__ double scratch[kDriftThreads / 32];
     __shared__ int s_refresh;
     double acc[4] = {0, 0, 0, 0};

@@ -2,7 +2,7 @@
 // Head-Wise Adaptive Sparse Attention, abstract: online top-p sparse attention with
 // per-head thresholds).
 //
-// One CTA per (query block i, head h). The row's scores become 64-bit keys
+// CTAs walk (head, query block) rows. A row's scores become 64-bit keys
 // (~float_bits << 32 | j) so that one ascending bitonic sort in shared memory orders them
 // by score descending, then index ascending. A block-wide float32 inclusive scan of the
 // sorted scores finds the first position whose cumulative mass reaches p; the kept set is
@@ -31,11 +31,13 @@ __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
     __shared__ int warp_cnt[NT / 32];
     __shared__ int cut_pos;
 
-    const int i = blockIdx.x, h = blockIdx.y;
-    if (head_mask != nullptr && head_mask[h] == 0) return;
     const int nb = g.nb;
-    if (!sort_all && i < g.nbv && p[h] < 1.0f && cnt[(size_t)h * nb + i] != -1) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int rowi = blockIdx.x; rowi < g.heads * nb; rowi += gridDim.x) {
+    const int h = rowi / nb, i = rowi - h * nb;
+    if (head_mask != nullptr && head_mask[h] == 0) continue;
+    if (!sort_all && i < g.nbv && p[h] < 1.0f && cnt[(size_t)h * nb + i] != -1) continue;
+    __syncthreads();                       // the previous row is finished with shared memory
     const float* row = scores + ((size_t)h * nb + i) * nb;
 
     for (int e = tid; e < N2; e += NT) {
@@ -134,6 +136,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
         if (flags[e]) out[base++] = (int)(uint32_t)key[tid * E + e];
     }
     if (tid == 0) cnt[(size_t)h * nb + i] = total;
+    }
 }
 
 
