@@ -8,7 +8,7 @@
 
 #include "bsa_common.cuh"
 #include "score.cuh"
-#include "park.cuh"
+#include "park_tc.cuh"
 #include "select.cuh"
 #include "drift.cuh"
 #include "attention.cuh"
@@ -80,7 +80,42 @@ size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(i
 
 // Score workspace: [pooled Q means | pooled K means: heads*nb*d fp32 each][block-slot table]
 size_t pooled_bytes(const Geom& g) { return align256((size_t)2 * g.heads * g.nb * g.d * sizeof(float)); }
-size_t score_ws_bytes(const Geom& g) { return pooled_bytes(g) + perm_bytes(g); }
+int park_nbp(const Geom& g) { return (g.nb + park::NT - 1) / park::NT * park::NT; }
+// PARK also keeps the three bf16 parts of the pooled keys: [heads][3][nbp][d]
+size_t ksplit_bytes(const Geom& g) { return align256((size_t)g.heads * 3 * park_nbp(g) * g.d * 2); }
+size_t score_ws_bytes(const Geom& g, int mode) {
+    return pooled_bytes(g) + perm_bytes(g) + (mode == BSA_SCORE_PARK ? ksplit_bytes(g) : 0);
+}
+
+template <int D>
+int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* perm, const int* head_mask,
+                float* scores, bsa_bf16* ksplit, cudaStream_t st) {
+    using C = park::Cfg<D>;
+    const int nbp = park_nbp(g);
+    const long long n = (long long)g.heads * nbp * D;
+    park::split_kbar_kernel<D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(g, kbar, nbp, ksplit);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaFuncSetAttribute(park::park_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+        return BSA_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    park::Params P;
+    P.g = g;
+    P.Q = Q;
+    P.ksplit = ksplit;
+    P.perm = perm;
+    P.head_mask = head_mask;
+    P.scores = scores;
+    P.nbp = nbp;
+    P.n_items = g.heads * g.nb;
+    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    const int grid = P.n_items < sms ? P.n_items : sms;
+    park::park_tc_kernel<D><<<grid, park::kThreads, C::SMEM, st>>>(P);
+    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
 
 int drift_chunks(const Geom& g) {
     const long long elems = (long long)g.N * g.d;
@@ -155,7 +190,7 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.tile_t = g.tt;
     info.tile_h = g.th;
     info.tile_w = g.tw;
-    info.score_workspace_bytes = score_ws_bytes(g);
+    info.score_workspace_bytes = score_ws_bytes(g, prob->score_mode);
     info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
     info.attention_workspace_bytes = attention_ws_bytes(g);
     *out = info;
@@ -179,7 +214,7 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || scores == nullptr) return BSA_ERR_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
-    if (ws == nullptr || ws_bytes < score_ws_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (ws == nullptr || ws_bytes < score_ws_bytes(g, prob->score_mode)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* qbar = static_cast<float*>(ws);
@@ -216,7 +251,9 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
 #undef BSA_MP
         return launch_status();
     }
-    return launch_park(g, Q, kbar, head_mask, scores, st);
+    bsa_bf16* ksplit = reinterpret_cast<bsa_bf16*>(static_cast<uint8_t*>(ws) + pooled_bytes(g) + perm_bytes(g));
+    if (g.d == 128) return launch_park<128>(g, Q, kbar, perm, head_mask, scores, ksplit, st);
+    return launch_park<64>(g, Q, kbar, perm, head_mask, scores, ksplit, st);
 }
 
 int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p,
