@@ -8,13 +8,15 @@
 // log2-sum-exp) go to the workspace and are merged by merge_text_kernel. Text items come
 // first in the item order, so the long ones start early.
 //
-// Warp roles (352 threads):
-//   warps 0-7  softmax + epilogue. Warp w owns query rows 32*(w%4) .. +31 (its TMEM lane
-//              quarter) and column half w/4 of S, P and O. The two warps of a row group
-//              exchange their half-row maxima once per block (bounded mbarrier), then each
-//              writes P only over its own S columns.
-//   warp 8     TMEM allocation; one elected thread issues every tcgen05.mma.
-//   warps 9-10 loaders: gather Q / K / V rows of a block (raster rows from the block-slot
+// Warp roles (480 threads):
+//   warps 0-7  softmax: warp w owns query rows 32*(w%4) .. +31 (its TMEM lane quarter) and
+//              column half w/4 of S / P; the two warps of a quarter swap half-row maxima
+//              once per block (a short bounded spin on an mbarrier).
+//   warps 8-11 epilogue: once the MMA has committed an item's last PV, read O[item&1] out of
+//              TMEM, divide by the row sum and store the rows (bf16 O, or the text rows'
+//              float32 partials); also writes the rows of items with nothing kept.
+//   warp 12    TMEM allocation; one elected thread issues every tcgen05.mma.
+//   warps 13-14 loaders: gather Q / K / V rows of a block (raster rows from the block-slot
 //              table) with 16-byte cp.async into 128B-swizzled K-major tiles; completion
 //              arrives on the tile's mbarrier asynchronously.
 // The kept blocks of all items of a CTA form one stream g = 0, 1, 2, ...:
@@ -24,10 +26,9 @@
 //   grows by more than 2^8, so O (in TMEM) is rarely rescaled; P <= 2^8 fits bf16 and the
 //   final division by the row sum is exact either way.
 // S/P is double-buffered (QK^T of block g+1 overlaps the softmax of block g, and the
-// softmax of block g+1 overlaps PV of block g); Q and O are double-buffered across items
-// (the next item's loads and QK^T overlap this item's epilogue). Every wait is bounded: one that runs out raises BSA_ERR_TIMEOUT and all roles
-// wind down. tcgen05.ld/st are warp-collective, so every condition around them is
-// warp-uniform.
+// softmax of block g+1 overlaps PV of block g); Q, O, K and V are double-buffered. Every wait is bounded: one that runs out raises
+// BSA_ERR_TIMEOUT and all roles wind down. tcgen05.ld/st are warp-collective, so every
+// condition around them is warp-uniform.
 #pragma once
 
 #include "bsa_common.cuh"
@@ -36,12 +37,15 @@ namespace bsa {
 namespace attn {
 
 constexpr int BQ = 128;                 // query rows per tile (MMA M)
-constexpr int kSoftmaxThreads = 256;    // 8 warps: 2 per row group, each half the columns
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp0 = 9;
-constexpr int kLoadThreads = 64;        // 11 warps in all: at most 3 per SM sub-partition
-constexpr int kThreads = kSoftmaxThreads + 32 + kLoadThreads;   // 352
-constexpr int NS = 2;                   // K and V pipeline stages
+constexpr int kSoftmaxThreads = 256;    // 8 warps: 2 per TMEM lane quarter, a column half each
+constexpr int kEpiWarp0 = 8;
+constexpr int kEpiThreads = 128;
+constexpr int kMmaWarp = 12;
+constexpr int kLoadWarp0 = 13;
+constexpr int kLoadThreads = 64;
+constexpr int kThreads = kSoftmaxThreads + kEpiThreads + 32 + kLoadThreads;   // 480
+constexpr int NK = 2;                   // K pipeline stages
+constexpr int NV = 2;                   // V pipeline stages
 constexpr int kTextChunk = 64;          // kept blocks per work item of a text query row
 constexpr float kRescaleLog2 = 8.0f;    // O is rescaled only when a row max grows by > 2^8
 
@@ -50,18 +54,17 @@ struct Cfg {
     static constexpr int Q_BYTES = BQ * D * 2;
     static constexpr int KV_BYTES = BK * D * 2;
     static constexpr int OFF_Q = 0;                          // 2 buffers
-    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // NS stages
-    static constexpr int OFF_V = OFF_K + NS * KV_BYTES;      // NS stages
-    static constexpr int OFF_STAGE = OFF_V + NS * KV_BYTES;  // bf16 O rows of one item
-    static constexpr int OFF_STAGE_TOK = OFF_STAGE + BQ * D * 2;
-    // [2 slots][2 halves][BQ]: half-row maxima of a block (slot = block parity); during an
-    // epilogue the slot of the next block holds the two halves' row sums instead
-    static constexpr int OFF_PMAX = OFF_STAGE_TOK + BQ * 4;
-    static constexpr int OFF_BAR = OFF_PMAX + 4 * BQ * 4;
-    // q_full[2] q_empty[2] k_full[NS] v_full[NS] k_empty[NS] v_empty[NS] s_full[2] s_free[2]
-    // p_full pv_done o_free[2] fin stage  (s_free[b]: the PV that read P out of S buffer b is
-    // done; stage: the 128 softmax threads meet around the epilogue's staging tile)
-    static constexpr int NBAR = 4 + 4 * NS + 4 + 2 + 2 + 1 + 1 + 4;   // + pair[4]
+    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // NK stages
+    static constexpr int OFF_V = OFF_K + NK * KV_BYTES;      // NV stages
+    static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;     // [2 O buffers][m, l0, l1][BQ]
+    static constexpr int OFF_PMAX = OFF_ML + 2 * 3 * BQ * 4; // [2 blocks][2 halves][BQ] maxima
+    static constexpr int OFF_BAR = OFF_PMAX + 2 * 2 * BQ * 4;
+    // q_full[2] q_empty[2] k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] s_free[2]
+    // p_full pv_done o_full[2] ml_ready[2] o_free[2] fin
+    // (s_free[b]: the PV that read P out of S buffer b is done; o_full[b]: the item's last
+    // PV into O buffer b is done; ml_ready[b]: its row max and sum are in shared memory;
+    // o_free[b]: the epilogue has read O buffer b and its row max and sum)
+    static constexpr int NBAR = 4 + 2 * NK + 2 * NV + 4 + 2 + 6 + 1 + 4;   // + pair[4]
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 8;         // +8: TMEM address slot
     static constexpr int TMEM_S = 0;            // S buffers: [0, 2*BK); P (bf16 pairs) overwrites
                                                 // the first BK/2 columns of its S buffer
@@ -234,18 +237,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
     uint64_t* q_full = bars;
     uint64_t* q_empty = bars + 2;
     uint64_t* k_full = bars + 4;
-    uint64_t* v_full = k_full + NS;
-    uint64_t* k_empty = v_full + NS;
-    uint64_t* v_empty = k_empty + NS;
-    uint64_t* s_full = v_empty + NS;
+    uint64_t* k_empty = k_full + NK;
+    uint64_t* v_full = k_empty + NK;
+    uint64_t* v_empty = v_full + NV;
+    uint64_t* s_full = v_empty + NV;
     uint64_t* s_free = s_full + 2;
     uint64_t* p_full = s_free + 2;
     uint64_t* pv_done = p_full + 1;
-    uint64_t* o_free = pv_done + 1;
+    uint64_t* o_full = pv_done + 1;
+    uint64_t* ml_ready = o_full + 2;
+    uint64_t* o_free = ml_ready + 2;
     uint64_t* fin_bar = o_free + 2;
-    uint64_t* stage_bar = fin_bar + 1;
-    uint64_t* pair_bar = stage_bar + 1;   // [4]: the two warps of a TMEM lane quarter
+    uint64_t* pair_bar = fin_bar + 1;   // [4]: the two softmax warps of a TMEM lane quarter
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + C::NBAR * 8);
+    float* ml = reinterpret_cast<float*>(sm + C::OFF_ML);   // [ob][0: m, 1: l half 0, 2: l half 1][row]
+    float* pmax = reinterpret_cast<float*>(sm + C::OFF_PMAX);
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
@@ -257,18 +263,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
             mbar_init(&s_free[b], 1);
-            mbar_init(&o_free[b], kSoftmaxThreads);
+            mbar_init(&o_full[b], 1);
+            mbar_init(&ml_ready[b], kSoftmaxThreads);
+            mbar_init(&o_free[b], kEpiThreads);
         }
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NK; ++s) {
             mbar_init(&k_full[s], kLoadThreads);
-            mbar_init(&v_full[s], kLoadThreads);
             mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < NV; ++s) {
+            mbar_init(&v_full[s], kLoadThreads);
             mbar_init(&v_empty[s], 1);
         }
         mbar_init(p_full, kSoftmaxThreads);
         mbar_init(pv_done, 1);
         mbar_init(fin_bar, 1);
-        mbar_init(stage_bar, kSoftmaxThreads);
         for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
         fence_mbar_init();
     }
@@ -315,20 +324,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             gather_tile<D, BQ>(tq, P.Q + head_off, sQ + qb * C::Q_BYTES, lt);
             cp_async_arrive_noinc(&q_full[qb]);
             for (int j = 0; j < it.n && ok; ++j, ++gblk) {
-                const int s = gblk % NS;
+                const int ks = gblk % NK, vs = gblk % NV;
                 const RowToks<D, BK> cur = tk;
                 if (j + 1 < it.n) {          // prefetch: next block's tokens, index two ahead
                     tk = load_tokens<D, BK>(P, kb_ahead, lt);
                     if (j + 2 < it.n) kb_ahead = kept_block(it, j + 2);
                 }
-                if (gblk >= NS) ok = mbar_wait(&k_empty[s], ((gblk / NS) - 1) & 1);
+                if (gblk >= NK) ok = mbar_wait(&k_empty[ks], ((gblk / NK) - 1) & 1);
                 if (!ok) break;
-                gather_tile<D, BK>(cur, P.K + head_off, sK + s * C::KV_BYTES, lt);
-                cp_async_arrive_noinc(&k_full[s]);
-                if (gblk >= NS) ok = mbar_wait(&v_empty[s], ((gblk / NS) - 1) & 1);
+                gather_tile<D, BK>(cur, P.K + head_off, sK + ks * C::KV_BYTES, lt);
+                cp_async_arrive_noinc(&k_full[ks]);
+                if (gblk >= NV) ok = mbar_wait(&v_empty[vs], ((gblk / NV) - 1) & 1);
                 if (!ok) break;
-                gather_tile<D, BK>(cur, P.V + head_off, sV + s * C::KV_BYTES, lt);
-                cp_async_arrive_noinc(&v_full[s]);
+                gather_tile<D, BK>(cur, P.V + head_off, sV + vs * C::KV_BYTES, lt);
+                cp_async_arrive_noinc(&v_full[vs]);
             }
             ++k;
         }
@@ -338,15 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
         if (elect_one()) {
             bool ok = true;
             // PV for stream block gb, the j-th block of the item with local index kitem. P is
-            // read from the first BK/4 columns of each column half of S buffer gb&1: key k of
-            // half h sits at column h*BK/2 + (k - h*BK/2)/2.
-            auto issue_pv = [&](int gb, int j, int kitem) -> bool {
+            // read from S buffer gb&1: the keys of column half h were packed into the first
+            // BK/4 columns of that half's region (key k of half h at column
+            // h*BK/2 + (k - h*BK/2)/2), 8 columns per 16 keys.
+            auto issue_pv = [&](int gb, int j, int kitem, bool last) -> bool {
                 const int ob = kitem & 1;
                 if (j == 0 && kitem >= 2 && !mbar_wait(&o_free[ob], ((kitem >> 1) - 1) & 1)) return false;
                 if (!mbar_wait(p_full, gb & 1)) return false;
-                if (!mbar_wait(&v_full[gb % NS], (gb / NS) & 1)) return false;
+                if (!mbar_wait(&v_full[gb % NV], (gb / NV) & 1)) return false;
                 tc_fence_after();
-                const uint32_t vbase = sV + (gb % NS) * C::KV_BYTES;
+                const uint32_t vbase = sV + (gb % NV) * C::KV_BYTES;
                 const uint32_t pcol = tmem + C::TMEM_S + (gb & 1) * BK;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
@@ -358,24 +368,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 }
                 tc_commit(pv_done);
                 tc_commit(&s_free[gb & 1]);
-                tc_commit(&v_empty[gb % NS]);
+                tc_commit(&v_empty[gb % NV]);
+                if (last) tc_commit(&o_full[ob]);
                 return true;
             };
             int gblk = 0, k = 0;
             int prev_g = -1, prev_j = 0, prev_k = 0;
+            bool prev_last = false;
             for (int item = first_item; item < P.n_items && ok; item += stride) {
                 const Item it = decode_item(P, item);
                 if (it.n <= 0) continue;
                 const int qb = k & 1;
                 ok = mbar_wait(&q_full[qb], (k >> 1) & 1);
                 for (int j = 0; j < it.n && ok; ++j, ++gblk) {
-                    const int s = gblk % NS, sb = gblk & 1;
-                    ok = mbar_wait(&k_full[s], (gblk / NS) & 1);
+                    const int ks = gblk % NK, sb = gblk & 1;
+                    ok = mbar_wait(&k_full[ks], (gblk / NK) & 1);
                     if (ok && gblk >= 2) ok = mbar_wait(&s_free[sb], ((gblk >> 1) - 1) & 1);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t qbase = sQ + qb * C::Q_BYTES;
-                    const uint32_t kbase = sK + s * C::KV_BYTES;
+                    const uint32_t kbase = sK + ks * C::KV_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = smem_desc_sw128(qbase + (kk >> 2) * C::Q_PANEL + (kk & 3) * 32, 16, 1024);
@@ -383,156 +395,37 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                         mma_bf16_ss(tmem + C::TMEM_S + sb * BK, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&s_full[sb]);
-                    tc_commit(&k_empty[s]);
+                    tc_commit(&k_empty[ks]);
                     if (j == it.n - 1) tc_commit(&q_empty[qb]);
-                    if (prev_g >= 0) ok = issue_pv(prev_g, prev_j, prev_k);
+                    if (prev_g >= 0) ok = issue_pv(prev_g, prev_j, prev_k, prev_last);
                     prev_g = gblk;
                     prev_j = j;
                     prev_k = k;
+                    prev_last = (j == it.n - 1);
                 }
                 ++k;
             }
-            if (ok && prev_g >= 0) ok = issue_pv(prev_g, prev_j, prev_k);
+            if (ok && prev_g >= 0) ok = issue_pv(prev_g, prev_j, prev_k, prev_last);
             // every MMA issued by this thread has completed once fin_bar flips
             tc_commit(fin_bar);
             mbar_wait(fin_bar, 0);
         }
         __syncwarp();
-    } else {
-        // ================================================================ softmax
+    } else if (warp < kEpiWarp0) {
         const int lane = threadIdx.x & 31;
         const int quarter = warp & 3;                    // TMEM lane quarter
-        const int half = warp >> 2;                      // column half of S / P / O
+        const int half = warp >> 2;                      // column half of S / P
         const int r = quarter * 32 + lane;               // query row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        constexpr int HB = BK / 2;                       // S / P columns of a half (keys)
-        constexpr int HD = D / 2;                        // O columns of a half
-        constexpr int CH = D / 8;                        // 16-byte chunks per O row
-        const uint32_t s_stage = smem_u32(sm + C::OFF_STAGE);
-        int* stage_tok = reinterpret_cast<int*>(sm + C::OFF_STAGE_TOK);
-        float* pmax = reinterpret_cast<float*>(sm + C::OFF_PMAX);
+        constexpr int HB = BK / 2;                       // keys of a column half
         bool ok = true;
-        uint32_t pair_phase = 0;
         int gblk = 0, k = 0;
-
-        // The epilogue of a finished item is deferred until the next item's first block has
-        // been handed to the MMA, so the item's last PV runs while that block is processed.
-        struct Pending {
-            bool active, split;
-            int item, h, q_token, ob;
-            float m, l;                                  // l: this half's partial row sum
-        };
-        Pending pend;
-        pend.active = false;
-
-        // all softmax threads meet here (bounded: a wait that runs out returns false)
-        uint32_t stage_phase = 0;
-        auto stage_sync = [&]() -> bool {
-            mbar_arrive(stage_bar);
-            const bool done = mbar_wait(stage_bar, stage_phase & 1);
-            ++stage_phase;
-            return __all_sync(0xffffffffu, done);
-        };
-
-        // gnext: index of the next block in the stream; its max-exchange slot is idle now
-        auto epilogue = [&](const Pending& pe, int gnext) -> bool {
-            const uint32_t o_col = lane_base + C::TMEM_O + pe.ob * D + half * HD;
-            float* lsum = pmax + (gnext & 1) * 2 * BQ;
-            // row sum: the two halves' partial sums meet in shared memory
-            if (!stage_sync()) return false;         // previous epilogue done with the tile
-            lsum[half * BQ + r] = pe.l;
-            if (half == 0) stage_tok[r] = pe.split ? -1 : pe.q_token;
-            uint32_t t0[32], t1[32];
-            tmem_ld32(o_col, t0);
-            if (HD > 32) tmem_ld32(o_col + 32, t1);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&o_free[pe.ob]);             // O has been read out of TMEM
-            if (!stage_sync()) return false;         // both halves of lsum are written
-            const float l = lsum[r] + lsum[BQ + r];
-            const float inv = 1.0f / l;
-            if (pe.split) {
-                float* po = P.part_o + ((size_t)pe.item * BQ + r) * D + half * HD;
-#pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(po + e) =
-                        make_float4(__uint_as_float(t0[e]) * inv, __uint_as_float(t0[e + 1]) * inv,
-                                    __uint_as_float(t0[e + 2]) * inv, __uint_as_float(t0[e + 3]) * inv);
-                if (HD > 32) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(po + 32 + e) =
-                            make_float4(__uint_as_float(t1[e]) * inv, __uint_as_float(t1[e + 1]) * inv,
-                                        __uint_as_float(t1[e + 2]) * inv, __uint_as_float(t1[e + 3]) * inv);
-                }
-                if (half == 0) P.part_lse[(size_t)pe.item * BQ + r] = pe.m + __log2f(l);
-                return stage_sync();                 // lsum slot read by every thread
-            }
-            // bf16 rows into the staging tile: 16-byte chunk c of row r at slot c ^ (r % CH)
-#pragma unroll
-            for (int u = 0; u < HD / 8; ++u) {
-                const uint32_t* t = u < 4 ? t0 : t1;
-                const int e0 = (u & 3) * 8;
-                uint32_t pk[4];
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(t[e0 + 2 * v]) * inv,
-                                                              __uint_as_float(t[e0 + 2 * v + 1]) * inv);
-                    pk[v] = *reinterpret_cast<uint32_t*>(&b2);
-                }
-                const int chunk = half * (HD / 8) + u;
-                const uint32_t dst = s_stage + r * (D * 2) + ((chunk ^ (r & (CH - 1))) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
-                             "r"(pk[2]), "r"(pk[3]) : "memory");
-            }
-            if (!stage_sync()) return false;         // the tile is complete
-            // coalesced write-out: warp w writes rows 16w .. 16w+15, CH lanes per row
-            bsa_bf16* Oh = P.O + (size_t)pe.h * g.N * D;
-            constexpr int RPI = 32 / CH;             // rows per instruction
-            constexpr int NIT = 16 / RPI;
-            const int cc = lane % CH;
-            uint4 v[NIT];
-            int tok[NIT];
-#pragma unroll
-            for (int q = 0; q < NIT; ++q) {
-                const int R = warp * 16 + q * RPI + lane / CH;
-                tok[q] = stage_tok[R];
-                const uint32_t src = s_stage + R * (D * 2) + ((cc ^ (R & (CH - 1))) << 4);
-                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(v[q].x), "=r"(v[q].y), "=r"(v[q].z), "=r"(v[q].w) : "r"(src));
-            }
-#pragma unroll
-            for (int q = 0; q < NIT; ++q)
-                if (tok[q] >= 0) *reinterpret_cast<uint4*>(Oh + (size_t)tok[q] * D + cc * 8) = v[q];
-            return true;
-        };
-
-        int item = first_item;
-        Item it;
-        if (item < P.n_items) it = decode_item(P, item);
-        while (item < P.n_items && ok) {
-            const int next_item = item + stride;
-            Item nxt;
-            if (next_item < P.n_items) nxt = decode_item(P, next_item);   // prefetched
-            const size_t head_off = (size_t)it.h * g.N * D;
-            const int q_token = (r < g.B) ? __ldg(P.perm + it.i * g.B + r) : -1;
-            if (it.n <= 0) {
-                // nothing kept (an empty text chunk, or an invalid count): zero output
-                if (it.n < 0 && threadIdx.x == 0) raise_error(BSA_ERR_DEVICE_ARG);
-                if (it.split) {
-                    float* po = P.part_o + ((size_t)item * BQ + r) * D + half * HD;
-                    for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(po + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (half == 0) P.part_lse[(size_t)item * BQ + r] = -INFINITY;
-                } else if (q_token >= 0) {
-                    bsa_bf16* orow = P.O + head_off + (size_t)q_token * D + half * HD;
-                    for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-                }
-                item = next_item;
-                it = nxt;
-                continue;
-            }
+        uint32_t pair_phase = 0;
+        for (int item = first_item; item < P.n_items && ok; item += stride) {
+            const Item it = decode_item(P, item);
+            if (it.n <= 0) continue;                     // the epilogue warps write zeros
             const int ob = k & 1;
-            const uint32_t o_col = lane_base + C::TMEM_O + ob * D + half * HD;
+            const uint32_t o_col = lane_base + C::TMEM_O + ob * D + half * (D / 2);
             float m = -INFINITY, l = 0.f;   // reference max (log2 units), this half's row sum
             int kb_next = kept_block(it, 0);
             for (int j = 0; j < it.n && ok; ++j, ++gblk) {
@@ -543,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (gblk >> 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
-                // pass 1: max of this half's raw scores (padding keys excluded), then the two
-                // halves of the row swap maxima so both use the same reference max
+                // pass 1: max of this half's raw scores (padding keys excluded); the two halves
+                // of a row then swap maxima so both use the same reference max
                 float mx = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < HB / 32; ++c) {
@@ -565,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                     float* slot = pmax + (gblk & 1) * 2 * BQ;
                     slot[half * BQ + r] = mx;
                     mbar_arrive(&pair_bar[quarter]);
-                    ok = __all_sync(0xffffffffu, mbar_wait(&pair_bar[quarter], pair_phase & 1));
+                    ok = __all_sync(0xffffffffu, mbar_wait_spin(&pair_bar[quarter], pair_phase & 1));
                     ++pair_phase;
                     if (!ok) break;
                     mx = fmaxf(mx, slot[(half ^ 1) * BQ + r]);
@@ -584,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 unsigned long long sum2 = pack2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < HB / 32; ++c) {
-                    const int key0 = half * HB + c * 32;         // first key of this chunk
+                    const int key0 = half * HB + c * 32;
                     uint32_t t[32];
                     tmem_ld32(s_col + key0, t);
                     tmem_wait_ld();
@@ -604,24 +497,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                         pk[e] = *reinterpret_cast<uint32_t*>(&b2);
                         sum2 = add2(sum2, pack2(p0, p1));
                     }
-                    // keys [key0, key0+32) -> P columns half*HB + (key0 - half*HB)/2 + [0,16),
+                    // keys [key0, key0+32) of half h -> P columns h*HB + (key0 - h*HB)/2 + [0,16),
                     // inside this half's S region and already read
                     tmem_st16(s_col + half * HB + (key0 - half * HB) / 2, pk);
                 }
                 const float2 sum = unpack2(sum2);
-                const float rs = sum.x + sum.y;
-                l = l * alpha + rs;
-                if (j >= 1 || pend.active) {
-                    // the previous PV (this item's, or the pending item's last) must be done
-                    // before O may be rescaled or PV of this block is issued; every PV is
-                    // waited for here, in order
+                l = l * alpha + (sum.x + sum.y);
+                if (gblk >= 1) {
+                    // the previous PV must be done before O may be rescaled or PV of this
+                    // block is issued; every PV is waited for here, in order
                     ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (gblk - 1) & 1));
                     if (!ok) break;
                     tc_fence_after();
                     // the whole warp takes part when any of its rows moved its reference max
                     if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-                        for (int c = 0; c < HD / 32; ++c) {
+                        for (int c = 0; c < D / 64; ++c) {
                             uint32_t t[32];
                             tmem_ld32(o_col + c * 32, t);
                             tmem_wait_ld();
@@ -634,30 +525,95 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(p_full);
-                if (j == 0 && pend.active) {
-                    ok = epilogue(pend, gblk + 1);
-                    pend.active = false;
-                }
             }
             if (!ok) break;
-            pend.active = true;
-            pend.split = it.split;
-            pend.item = item;
-            pend.h = it.h;
-            pend.q_token = q_token;
-            pend.ob = ob;
-            pend.m = m;
-            pend.l = l;
+            // hand the row max and this half's row sum to the epilogue; O buffer ob (and its
+            // m, l slots) must have been released by the epilogue of the item two back
+            if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((k >> 1) - 1) & 1));
+            if (!ok) break;
+            if (half == 0) ml[(ob * 3 + 0) * BQ + r] = m;
+            ml[(ob * 3 + 1 + half) * BQ + r] = l;
+            mbar_arrive(&ml_ready[ob]);
             ++k;
+        }
+    } else if (warp < kMmaWarp) {
+        // ================================================================ epilogue
+        const int quarter = warp - kEpiWarp0;
+        const int r = quarter * 32 + (threadIdx.x & 31);  // query row == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        bool ok = true;
+        int k = 0;
+        int item = first_item;
+        Item it;
+        if (item < P.n_items) it = decode_item(P, item);
+        while (item < P.n_items && ok) {
+            const int next_item = item + stride;
+            Item nxt;
+            if (next_item < P.n_items) nxt = decode_item(P, next_item);   // prefetched
+            const size_t head_off = (size_t)it.h * g.N * D;
+            const int q_token = (r < g.B) ? __ldg(P.perm + it.i * g.B + r) : -1;
+            if (it.n <= 0) {
+                // nothing kept (an empty text chunk, or an invalid count): zero output
+                if (it.n < 0 && r == 0) raise_error(BSA_ERR_DEVICE_ARG);
+                if (it.split) {
+                    float* po = P.part_o + ((size_t)item * BQ + r) * D;
+                    for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(po + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    P.part_lse[(size_t)item * BQ + r] = -INFINITY;
+                } else if (q_token >= 0) {
+                    bsa_bf16* orow = P.O + head_off + (size_t)q_token * D;
+                    for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                }
+            } else {
+                const int ob = k & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (k >> 1) & 1));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ml_ready[ob], (k >> 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+                const float m = ml[(ob * 3 + 0) * BQ + r];
+                const float l = ml[(ob * 3 + 1) * BQ + r] + ml[(ob * 3 + 2) * BQ + r];
+                const float inv = 1.0f / l;
+                const uint32_t o_col = lane_base + C::TMEM_O + ob * D;
+                if (it.split) {
+                    float* po = P.part_o + ((size_t)item * BQ + r) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t t[32];
+                        tmem_ld32(o_col + c * 32, t);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4*>(po + c * 32 + e) =
+                                make_float4(__uint_as_float(t[e]) * inv, __uint_as_float(t[e + 1]) * inv,
+                                            __uint_as_float(t[e + 2]) * inv, __uint_as_float(t[e + 3]) * inv);
+                    }
+                    P.part_lse[(size_t)item * BQ + r] = m + __log2f(l);
+                } else {
+                    bsa_bf16* orow = P.O + head_off + (size_t)(q_token >= 0 ? q_token : 0) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t t[32];
+                        tmem_ld32(o_col + c * 32, t);
+                        tmem_wait_ld();
+                        if (q_token < 0) continue;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(t[e + 2 * u]) * inv,
+                                                                          __uint_as_float(t[e + 2 * u + 1]) * inv);
+                                pk[u] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&o_free[ob]);            // O buffer and its m, l are free again
+                ++k;
+            }
             item = next_item;
             it = nxt;
-        }
-        if (ok && pend.active) {
-            ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (gblk - 1) & 1));
-            if (ok) {
-                tc_fence_after();
-                ok = epilogue(pend, gblk);
-            }
         }
     }
 

@@ -130,6 +130,17 @@ __device__ inline bool mbar_test(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Bounded spin on a phase that is expected to complete within a few hundred cycles (two
+// warps meeting); no suspension, so the wake-up is immediate.
+__device__ inline bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity)) {
+        if (error_raised()) return false;
+        if (clock64() - t0 > kWaitLimitCycles) { raise_error(BSA_ERR_TIMEOUT); return false; }
+    }
+    return true;
+}
+
 // Wait for the phase with the given parity to complete. Gives up (raising
 // BSA_ERR_TIMEOUT) after kWaitLimitCycles or as soon as another thread raised an error.
 __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
