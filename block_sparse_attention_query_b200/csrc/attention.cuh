@@ -9,9 +9,12 @@
 // first in the item order, so the long ones start early.
 //
 // Warp roles (480 threads):
-//   warps 0-7  softmax: warp w owns query rows 32*(w%4) .. +31 (its TMEM lane quarter) and
-//              column half w/4 of S / P; the two warps of a quarter swap half-row maxima
-//              once per block (a short bounded spin on an mbarrier).
+//   warps 0-7  softmax, two groups of four warps. Group G takes the blocks g of the stream
+//              with g%2 == G, so the two groups work on consecutive blocks at the same time
+//              (one in its exponentials while the other reads and reduces its scores);
+//              warp w owns query rows 32*(w%4) .. +31 (its TMEM lane quarter), whole rows.
+//              The reference max of a row is chained from block to block through shared
+//              memory (a light dependency on the other group's first pass only).
 //   warps 8-11 epilogue: once the MMA has committed an item's last PV, read O[item&1] out of
 //              TMEM, divide by the row sum and store the rows (bf16 O, or the text rows'
 //              float32 partials); also writes the rows of items with nothing kept.
@@ -25,8 +28,9 @@
 //   TMEM (V is an MN-major smem operand). The reference max m only moves when a row max
 //   grows by more than 2^8, so O (in TMEM) is rarely rescaled; P <= 2^8 fits bf16 and the
 //   final division by the row sum is exact either way.
-// S/P is double-buffered (QK^T of block g+1 overlaps the softmax of block g, and the
-// softmax of block g+1 overlaps PV of block g); Q, O, K and V are double-buffered. Every wait is bounded: one that runs out raises
+// S/P is double-buffered (buffer g&1 belongs to softmax group g&1); Q, O, K and V are
+// double-buffered. Each group keeps its row sum relative to its own latest reference max; the
+// epilogue combines the two. Every wait is bounded: one that runs out raises
 // BSA_ERR_TIMEOUT and all roles wind down. tcgen05.ld/st are warp-collective, so every
 // condition around them is warp-uniform.
 #pragma once
@@ -37,7 +41,8 @@ namespace bsa {
 namespace attn {
 
 constexpr int BQ = 128;                 // query rows per tile (MMA M)
-constexpr int kSoftmaxThreads = 256;    // 8 warps: 2 per TMEM lane quarter, a column half each
+constexpr int kSoftmaxThreads = 256;    // 8 warps: 2 groups of 4 (one per TMEM lane quarter)
+constexpr int kGroupThreads = 128;
 constexpr int kEpiWarp0 = 8;
 constexpr int kEpiThreads = 128;
 constexpr int kMmaWarp = 12;
@@ -56,18 +61,19 @@ struct Cfg {
     static constexpr int OFF_Q = 0;                          // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // NK stages
     static constexpr int OFF_V = OFF_K + NK * KV_BYTES;      // NV stages
-    static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;     // [2 O buffers][m, l0, l1][BQ]
-    static constexpr int OFF_PMAX = OFF_ML + 2 * 3 * BQ * 4; // [2 blocks][2 halves][BQ] maxima
-    static constexpr int OFF_BAR = OFF_PMAX + 2 * 2 * BQ * 4;
+    static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;     // [2 O buffers][m0, l0, m1, l1][BQ]
+    static constexpr int OFF_MCH = OFF_ML + 2 * 4 * BQ * 4;  // [2 S buffers][BQ] chained maxima
+    static constexpr int OFF_BAR = OFF_MCH + 2 * BQ * 4;
     // q_full[2] q_empty[2] k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] s_free[2]
-    // p_full pv_done o_full[2] ml_ready[2] o_free[2] fin
+    // p_full[2] pv_done o_full[2] ml_ready[2] o_free[2] fin m_ready[2]
     // (s_free[b]: the PV that read P out of S buffer b is done; o_full[b]: the item's last
-    // PV into O buffer b is done; ml_ready[b]: its row max and sum are in shared memory;
-    // o_free[b]: the epilogue has read O buffer b and its row max and sum)
-    static constexpr int NBAR = 4 + 2 * NK + 2 * NV + 4 + 2 + 6 + 1 + 4;   // + pair[4]
+    // PV into O buffer b is done; ml_ready[b]: both groups' row max and sum are in shared
+    // memory; o_free[b]: the epilogue has read O buffer b and its row maxima and sums;
+    // m_ready[b]: the reference max of the latest block of S buffer b is published)
+    static constexpr int NBAR = 4 + 2 * NK + 2 * NV + 4 + 2 + 1 + 6 + 1 + 2;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 8;         // +8: TMEM address slot
-    static constexpr int TMEM_S = 0;            // S buffers: [0, 2*BK); P (bf16 pairs) overwrites
-                                                // the first BK/2 columns of its S buffer
+    static constexpr int TMEM_S = 0;            // S buffers: [0, 2*BK); P (bf16 pairs, key k at
+                                                // column k/2) overwrites the first BK/2 columns
     static constexpr int TMEM_O = 2 * BK;       // O buffers: [2*BK, 2*BK + 2*D)
     static constexpr int TMEM_COLS = (2 * BK + 2 * D) <= 256 ? 256 : 512;
     static constexpr int Q_PANEL = BQ * 128;    // bytes per 64-column swizzle panel
@@ -130,22 +136,6 @@ __device__ inline float max3(float a, float b, float c) {
     return d;
 }
 
-// 2^x on the FMA pipe, for x <= 8 (larger x is never passed here). Range reduction x = n + f
-// with n = round(x) by the 1.5*2^23 magic-constant add, f in [-0.5, 0.5]; 2^f from a degree-3
-// polynomial fitted by relative-error-weighted least squares (Lawson iterations) at Chebyshev
-// nodes of [-0.5, 0.5]; then n is added to the exponent field. Max relative error 7.5e-5 for
-// x >= -125 (well under the 2^-9 of the bf16 that P is rounded to); x below -125 is clamped
-// there (2^-125 ~ 2.4e-38 stands in for 0, and keeps the exponent field normal).
-__device__ inline float exp2_fma(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;            // 1.5 * 2^23: low mantissa bits hold round(x)
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(0.0551716648042202f, f, 0.2426111251115799f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999280571937561f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packed float32 pairs (fma.rn.f32x2 / add.rn.f32x2 run both lanes in one instruction).
 __device__ inline unsigned long long pack2(float a, float b) {
     unsigned long long r;
@@ -166,6 +156,43 @@ __device__ inline unsigned long long add2(unsigned long long a, unsigned long lo
     unsigned long long d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+
+// 2^x on the FMA pipe, for x <= 8 (larger x is never passed here). Range reduction x = n + f
+// with n = round(x) by the 1.5*2^23 magic-constant add, f in [-0.5, 0.5]; 2^f from a degree-3
+// polynomial fitted by relative-error-weighted least squares (Lawson iterations) at Chebyshev
+// nodes of [-0.5, 0.5]; then n is added to the exponent field. Max relative error 7.5e-5 for
+// x >= -125 (well under the 2^-9 of the bf16 that P is rounded to); x below -125 is clamped
+// there (2^-125 ~ 2.4e-38 stands in for 0, and keeps the exponent field normal).
+constexpr float kExp2Clamp = -125.0f;
+constexpr float kExp2Magic = 12582912.0f;     // 1.5 * 2^23: low mantissa bits hold round(x)
+constexpr float kExp2C3 = 0.0551716648042202f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C0 = 0.9999280571937561f;
+
+__device__ inline float exp2_fma(float x) {
+    x = fmaxf(x, kExp2Clamp);
+    const float t = x + kExp2Magic;
+    const float f = x - (t - kExp2Magic);
+    float p = fmaf(kExp2C3, f, kExp2C2);
+    p = fmaf(p, f, kExp2C1);
+    p = fmaf(p, f, kExp2C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same function on a pair, in packed float32x2 arithmetic (bit-identical results).
+__device__ inline float2 exp2_fma_pair(float2 x) {
+    const unsigned long long xx = pack2(fmaxf(x.x, kExp2Clamp), fmaxf(x.y, kExp2Clamp));
+    const unsigned long long t = add2(xx, pack2(kExp2Magic, kExp2Magic));
+    const unsigned long long n = add2(t, pack2(-kExp2Magic, -kExp2Magic));   // round(x), exact
+    const unsigned long long f = fma2(n, pack2(-1.0f, -1.0f), xx);           // x - round(x), exact
+    unsigned long long p = fma2(pack2(kExp2C3, kExp2C3), f, pack2(kExp2C2, kExp2C2));
+    p = fma2(p, f, pack2(kExp2C1, kExp2C1));
+    p = fma2(p, f, pack2(kExp2C0, kExp2C0));
+    const float2 pv = unpack2(p), tv = unpack2(t);
+    return make_float2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
+                       __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
 }
 
 // Pairs e (of 16 per 32 keys) whose exponentials run on the FMA pipe instead of the MUFU:
@@ -243,15 +270,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
     uint64_t* s_full = v_empty + NV;
     uint64_t* s_free = s_full + 2;
     uint64_t* p_full = s_free + 2;
-    uint64_t* pv_done = p_full + 1;
+    uint64_t* pv_done = p_full + 2;
     uint64_t* o_full = pv_done + 1;
     uint64_t* ml_ready = o_full + 2;
     uint64_t* o_free = ml_ready + 2;
     uint64_t* fin_bar = o_free + 2;
-    uint64_t* pair_bar = fin_bar + 1;   // [4]: the two softmax warps of a TMEM lane quarter
+    uint64_t* m_ready = fin_bar + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + C::NBAR * 8);
-    float* ml = reinterpret_cast<float*>(sm + C::OFF_ML);   // [ob][0: m, 1: l half 0, 2: l half 1][row]
-    float* pmax = reinterpret_cast<float*>(sm + C::OFF_PMAX);
+    float* ml = reinterpret_cast<float*>(sm + C::OFF_ML);     // [ob][m0, l0, m1, l1][row]
+    float* mch = reinterpret_cast<float*>(sm + C::OFF_MCH);   // [S buffer][row]
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
@@ -275,10 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             mbar_init(&v_full[s], kLoadThreads);
             mbar_init(&v_empty[s], 1);
         }
-        mbar_init(p_full, kSoftmaxThreads);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&p_full[b], kGroupThreads);
+            mbar_init(&m_ready[b], kGroupThreads);
+        }
         mbar_init(pv_done, 1);
         mbar_init(fin_bar, 1);
-        for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
@@ -347,23 +376,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
         if (elect_one()) {
             bool ok = true;
             // PV for stream block gb, the j-th block of the item with local index kitem. P is
-            // read from S buffer gb&1: the keys of column half h were packed into the first
-            // BK/4 columns of that half's region (key k of half h at column
-            // h*BK/2 + (k - h*BK/2)/2), 8 columns per 16 keys.
+            // read from S buffer gb&1 (key k at column k/2: 8 columns per 16 keys).
             auto issue_pv = [&](int gb, int j, int kitem, bool last) -> bool {
                 const int ob = kitem & 1;
                 if (j == 0 && kitem >= 2 && !mbar_wait(&o_free[ob], ((kitem >> 1) - 1) & 1)) return false;
-                if (!mbar_wait(p_full, gb & 1)) return false;
+                if (!mbar_wait(&p_full[gb & 1], (gb >> 1) & 1)) return false;
                 if (!mbar_wait(&v_full[gb % NV], (gb / NV) & 1)) return false;
                 tc_fence_after();
                 const uint32_t vbase = sV + (gb % NV) * C::KV_BYTES;
                 const uint32_t pcol = tmem + C::TMEM_S + (gb & 1) * BK;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
-                    const int hk = kk / (BK / 32);
-                    const uint32_t acol = kk * 8 + hk * (BK / 4);
                     const uint64_t b = smem_desc_sw128(vbase + kk * 2048, C::KV_PANEL, 1024);
-                    mma_bf16_ts(tmem + C::TMEM_O + ob * D, pcol + acol, b, C::IDESC_PV,
+                    mma_bf16_ts(tmem + C::TMEM_O + ob * D, pcol + kk * 8, b, C::IDESC_PV,
                                 (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(pv_done);
@@ -412,38 +437,38 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
         }
         __syncwarp();
     } else if (warp < kEpiWarp0) {
+        // ================================================================ softmax
         const int lane = threadIdx.x & 31;
         const int quarter = warp & 3;                    // TMEM lane quarter
-        const int half = warp >> 2;                      // column half of S / P
+        const int grp = warp >> 2;                       // owns the blocks g with g%2 == grp
         const int r = quarter * 32 + lane;               // query row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        constexpr int HB = BK / 2;                       // keys of a column half
+        const uint32_t s_col = lane_base + C::TMEM_S + grp * BK;
+        const unsigned long long scale2 = pack2(P.scale_log2, P.scale_log2);
         bool ok = true;
         int gblk = 0, k = 0;
-        uint32_t pair_phase = 0;
         for (int item = first_item; item < P.n_items && ok; item += stride) {
             const Item it = decode_item(P, item);
             if (it.n <= 0) continue;                     // the epilogue warps write zeros
             const int ob = k & 1;
-            const uint32_t o_col = lane_base + C::TMEM_O + ob * D + half * (D / 2);
-            float m = -INFINITY, l = 0.f;   // reference max (log2 units), this half's row sum
-            int kb_next = kept_block(it, 0);
-            for (int j = 0; j < it.n && ok; ++j, ++gblk) {
-                const int sb = gblk & 1;
-                const uint32_t s_col = lane_base + C::TMEM_S + sb * BK;
-                const int kcount = block_count(g, kb_next);
-                if (j + 1 < it.n) kb_next = kept_block(it, j + 1);   // prefetch for the next block
-                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (gblk >> 1) & 1));
+            const uint32_t o_col = lane_base + C::TMEM_O + ob * D;
+            // this group's reference max (log2 units) and row sum relative to it
+            float mref = -INFINITY, l = 0.f;
+            const int j0 = (gblk & 1) == grp ? 0 : 1;    // this group's first block of the item
+            int kb = j0 < it.n ? kept_block(it, j0) : 0;
+            for (int j = j0; j < it.n && ok; j += 2) {
+                const int g_cur = gblk + j;              // stream index of this block
+                const int kcount = block_count(g, kb);
+                if (j + 2 < it.n) kb = kept_block(it, j + 2);   // prefetch for the next block
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[grp], (g_cur >> 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
-                // pass 1: max of this half's raw scores (padding keys excluded); the two halves
-                // of a row then swap maxima so both use the same reference max
+                // pass 1: max of the row's raw scores (padding keys excluded)
                 float mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < HB / 32; ++c) {
-                    const int key0 = half * HB + c * 32;
+#pragma unroll 1
+                for (int c = 0; c < BK / 32; ++c) {
                     uint32_t t[32];
-                    tmem_ld32(s_col + key0, t);
+                    tmem_ld32(s_col + c * 32, t);
                     tmem_wait_ld();
                     if (kcount >= BK) {
 #pragma unroll
@@ -451,88 +476,93 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (key0 + e < kcount) mx = fmaxf(mx, __uint_as_float(t[e]));
+                            if (c * 32 + e < kcount) mx = fmaxf(mx, __uint_as_float(t[e]));
                     }
                 }
-                {
-                    float* slot = pmax + (gblk & 1) * 2 * BQ;
-                    slot[half * BQ + r] = mx;
-                    mbar_arrive(&pair_bar[quarter]);
-                    ok = __all_sync(0xffffffffu, mbar_wait_spin(&pair_bar[quarter], pair_phase & 1));
-                    ++pair_phase;
-                    if (!ok) break;
-                    mx = fmaxf(mx, slot[(half ^ 1) * BQ + r]);
-                }
                 const float m_blk = mx * P.scale_log2;
-                float alpha = 1.0f;
-                if (j == 0) {
-                    m = m_blk;
-                } else if (m_blk > m + kRescaleLog2) {
-                    alpha = ex2(m - m_blk);
-                    m = m_blk;
+                // reference max chain: block g takes the previous block's reference (published
+                // by the other group) and moves it only when its own max exceeds it by more
+                // than 2^8; the first block of an item starts afresh. Every block waits for
+                // its predecessor's entry, which keeps the two groups' entries in step.
+                float mprev = -INFINITY;
+                if (g_cur >= 1) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&m_ready[grp ^ 1], ((g_cur - 1) >> 1) & 1));
+                    if (!ok) break;
+                    mprev = mch[(grp ^ 1) * BQ + r];
                 }
-                // pass 2 on this half: P = 2^(s*scale - m) as bf16 pairs over the S columns
-                const unsigned long long scale2 = pack2(P.scale_log2, P.scale_log2);
+                const float m = (j == 0 || m_blk > mprev + kRescaleLog2) ? m_blk : mprev;
+                mch[grp * BQ + r] = m;
+                mbar_arrive(&m_ready[grp]);
+                // this group's sum follows its own reference
+                if (mref != -INFINITY && m != mref) l *= ex2(mref - m);
+                mref = m;
+                // pass 2: P = 2^(s*scale - m) as bf16 pairs, key k at column k/2 of the buffer
                 const unsigned long long negm2 = pack2(-m, -m);
                 unsigned long long sum2 = pack2(0.f, 0.f);
-#pragma unroll
-                for (int c = 0; c < HB / 32; ++c) {
-                    const int key0 = half * HB + c * 32;
+#pragma unroll 1
+                for (int c = 0; c < BK / 32; ++c) {
                     uint32_t t[32];
-                    tmem_ld32(s_col + key0, t);
+                    tmem_ld32(s_col + c * 32, t);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float2 x = unpack2(fma2(pack2(__uint_as_float(t[2 * e]), __uint_as_float(t[2 * e + 1])),
                                                       scale2, negm2));
-                        const bool soft = (BSA_SOFT_EXP_MASK >> (e % 8)) & 1;
-                        float p0 = soft ? exp2_fma(x.x) : ex2(x.x);
-                        float p1 = soft ? exp2_fma(x.y) : ex2(x.y);
+                        float p0, p1;
+                        if ((BSA_SOFT_EXP_MASK >> (e % 8)) & 1) {
+                            const float2 q = exp2_fma_pair(x);
+                            p0 = q.x;
+                            p1 = q.y;
+                        } else {
+                            p0 = ex2(x.x);
+                            p1 = ex2(x.y);
+                        }
                         if (kcount < BK) {
-                            if (key0 + 2 * e >= kcount) p0 = 0.f;
-                            if (key0 + 2 * e + 1 >= kcount) p1 = 0.f;
+                            if (c * 32 + 2 * e >= kcount) p0 = 0.f;
+                            if (c * 32 + 2 * e + 1 >= kcount) p1 = 0.f;
                         }
                         __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t*>(&b2);
                         sum2 = add2(sum2, pack2(p0, p1));
                     }
-                    // keys [key0, key0+32) of half h -> P columns h*HB + (key0 - h*HB)/2 + [0,16),
-                    // inside this half's S region and already read
-                    tmem_st16(s_col + half * HB + (key0 - half * HB) / 2, pk);
+                    // keys [32c, 32c+32) -> P columns [16c, 16c+16): S columns already read
+                    tmem_st16(s_col + c * 16, pk);
                 }
                 const float2 sum = unpack2(sum2);
-                l = l * alpha + (sum.x + sum.y);
-                if (gblk >= 1) {
-                    // the previous PV must be done before O may be rescaled or PV of this
-                    // block is issued; every PV is waited for here, in order
-                    ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (gblk - 1) & 1));
+                l += sum.x + sum.y;
+                // O holds the PVs of the blocks before this one at reference mprev: rescale it
+                // (whole warp, when any of its rows moved) once the previous PV is done.
+                // pv_done is at most one phase ahead of block g-1 here (S of this block was
+                // issued after the PV two blocks back completed, and PV of this block waits
+                // for p_full), so a parity wait is exact even though most blocks skip it.
+                if (j >= 1 && __any_sync(0xffffffffu, m != mprev)) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (g_cur - 1) & 1));
                     if (!ok) break;
                     tc_fence_after();
-                    // the whole warp takes part when any of its rows moved its reference max
-                    if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                    const float alpha = ex2(mprev - m);   // 1 for rows that kept their max
 #pragma unroll 1
-                        for (int c = 0; c < D / 64; ++c) {
-                            uint32_t t[32];
-                            tmem_ld32(o_col + c * 32, t);
-                            tmem_wait_ld();
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_col + c * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
-                            tmem_st32(o_col + c * 32, t);
-                        }
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(o_col + c * 32, o);
                     }
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                mbar_arrive(&p_full[grp]);
             }
             if (!ok) break;
-            // hand the row max and this half's row sum to the epilogue; O buffer ob (and its
-            // m, l slots) must have been released by the epilogue of the item two back
+            gblk += it.n;
+            // hand this group's reference max and row sum to the epilogue; O buffer ob (and
+            // its slots) must have been released by the epilogue of the item two back
             if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((k >> 1) - 1) & 1));
             if (!ok) break;
-            if (half == 0) ml[(ob * 3 + 0) * BQ + r] = m;
-            ml[(ob * 3 + 1 + half) * BQ + r] = l;
+            ml[(ob * 4 + 2 * grp) * BQ + r] = mref;
+            ml[(ob * 4 + 2 * grp + 1) * BQ + r] = l;
             mbar_arrive(&ml_ready[ob]);
             ++k;
         }
@@ -569,8 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ml_ready[ob], (k >> 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
-                const float m = ml[(ob * 3 + 0) * BQ + r];
-                const float l = ml[(ob * 3 + 1) * BQ + r] + ml[(ob * 3 + 2) * BQ + r];
+                // O is relative to the reference of the item's last block, the larger of the two
+                // groups' final references; each group's sum is relative to its own
+                const float m0 = ml[(ob * 4 + 0) * BQ + r], l0 = ml[(ob * 4 + 1) * BQ + r];
+                const float m1 = ml[(ob * 4 + 2) * BQ + r], l1 = ml[(ob * 4 + 3) * BQ + r];
+                const float m = fmaxf(m0, m1);
+                const float l = (l0 > 0.f ? l0 * ex2(m0 - m) : 0.f) + (l1 > 0.f ? l1 * ex2(m1 - m) : 0.f);
                 const float inv = 1.0f / l;
                 const uint32_t o_col = lane_base + C::TMEM_O + ob * D;
                 if (it.split) {

@@ -14,12 +14,12 @@ from tests.conftest import ROOT
 
 def _coeffs():
     src = open(os.path.join(ROOT, "block_sparse_attention_query_b200", "csrc", "attention.cuh")).read()
-    body = src[src.index("__device__ inline float exp2_fma"):]
-    body = body[:body.index("}")]
-    vals = [np.float32(v) for v in re.findall(r"([0-9]+\.[0-9]+)f", body)]
-    # clamp, magic constant twice, then the four polynomial coefficients (highest first)
-    assert vals[0] == np.float32(125.0) and vals[1] == vals[2] == np.float32(12582912.0)
-    return vals[3:7]
+    val = {}
+    for name in ("kExp2Clamp", "kExp2Magic", "kExp2C3", "kExp2C2", "kExp2C1", "kExp2C0"):
+        m = re.search(r"constexpr float " + name + r" = (-?[0-9]+\.[0-9]+)f;", src)
+        val[name] = np.float32(m.group(1))
+    assert val["kExp2Clamp"] == np.float32(-125.0) and val["kExp2Magic"] == np.float32(12582912.0)
+    return val["kExp2C3"], val["kExp2C2"], val["kExp2C1"], val["kExp2C0"]
 
 
 def _exp2_fma(x):
