@@ -63,7 +63,8 @@ struct Cfg {
     static constexpr int OFF_V = OFF_K + NK * KV_BYTES;      // NV stages
     static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;     // [2 O buffers][m0, l0, m1, l1][BQ]
     static constexpr int OFF_MCH = OFF_ML + 2 * 4 * BQ * 4;  // [2 S buffers][BQ] chained maxima
-    static constexpr int OFF_BAR = OFF_MCH + 2 * BQ * 4;
+    static constexpr int OFF_STG = OFF_MCH + 2 * BQ * 4;     // [4 epilogue warps][32 rows][128 B]
+    static constexpr int OFF_BAR = OFF_STG + 4 * 32 * 128;
     // q_full[2] q_empty[2] k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] s_free[2]
     // p_full[2] pv_done o_full[2] ml_ready[2] o_free[2] fin m_ready[2]
     // (s_free[b]: the PV that read P out of S buffer b is done; o_full[b]: the item's last
@@ -622,24 +623,41 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                     }
                     P.part_lse[(size_t)item * BQ + r] = m + __log2f(l);
                 } else {
-                    bsa_bf16* orow = P.O + head_off + (size_t)(q_token >= 0 ? q_token : 0) * D;
+                    // 64 columns at a time: the warp's 32 rows go through a 128B-swizzled staging
+                    // tile in shared memory so that each global store instruction writes four
+                    // whole 128-byte row segments
+                    const uint32_t stg = smem_u32(sm + C::OFF_STG) + (warp - kEpiWarp0) * 32 * 128;
+                    const int lane = threadIdx.x & 31;
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t t[32];
-                        tmem_ld32(o_col + c * 32, t);
-                        tmem_wait_ld();
-                        if (q_token < 0) continue;
+                    for (int hc = 0; hc < D / 64; ++hc) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint32_t pk[4];
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t t[32];
+                            tmem_ld32(o_col + hc * 64 + c * 32, t);
+                            tmem_wait_ld();
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(t[e + 2 * u]) * inv,
-                                                                          __uint_as_float(t[e + 2 * u + 1]) * inv);
-                                pk[u] = *reinterpret_cast<uint32_t*>(&b2);
+                            for (int e = 0; e < 32; e += 8) {
+                                uint32_t pk[4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(t[e + 2 * u]) * inv,
+                                                                              __uint_as_float(t[e + 2 * u + 1]) * inv);
+                                    pk[u] = *reinterpret_cast<uint32_t*>(&b2);
+                                }
+                                const int chunk = c * 4 + e / 8;
+                                st_shared_v4(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4), pk);
                             }
-                            *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int row = i * 4 + (lane >> 3), chunk = lane & 7;
+                            const int tok = __shfl_sync(0xffffffffu, q_token, row);
+                            const uint4 v = ld_shared_v4(stg + row * 128 + ((chunk ^ (row & 7)) << 4));
+                            if (tok >= 0)
+                                *reinterpret_cast<uint4*>(P.O + head_off + (size_t)tok * D + hc * 64 + chunk * 8) = v;
+                        }
+                        __syncwarp();
                     }
                 }
                 tc_fence_before();

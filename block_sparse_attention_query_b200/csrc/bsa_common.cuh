@@ -153,6 +153,18 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
     return true;
 }
 
+// 16-byte shared-memory accesses by address.
+__device__ inline void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+__device__ inline uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ PTX: cp.async
 
 __device__ inline void cp_async_16(uint32_t dst_smem, const void* src) {
