@@ -17,6 +17,7 @@ the calls all ranks made (ms per call, whole job).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -97,6 +98,27 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- ours
+
+def _profiled_traffic(kernel, workload):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, or None
+    when the kernel sources changed since that capture or the workload differs."""
+    if kernel != "sparse_attention":
+        return None
+    root = os.path.dirname(os.path.abspath(__file__))
+    prof = os.path.join(root, "profiles", f"sparse_attention_{workload}.md")
+    if not os.path.exists(prof):
+        return None
+    fields = {}
+    for line in open(prof):
+        k, sep, v = line.strip().partition(": ")
+        if sep and k in ("traffic_bytes_per_launch", "workload", "sources_sha256_16"):
+            fields[k] = v.strip()
+    src = b"".join(open(os.path.join(root, "block_sparse_attention_query_b200", "csrc", f), "rb").read()
+                   for f in ("attention.cuh", "bsa_common.cuh"))
+    if fields.get("workload") != workload or fields.get("sources_sha256_16") != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
 
 def run_ours(args, ws, rank, local):
     import torch
@@ -219,8 +241,11 @@ def run_ours(args, ws, rank, local):
         b = bytes_drift if dom == "drift_check" else bytes_score
         ach = b / (stage_ms[names.index(dom)] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4)}
+    traffic = args.traffic if args.traffic is not None else _profiled_traffic(dom, w.name)
     roof.update({"kernel": dom, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
-                 "traffic": args.traffic})
+                 "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
+                 "algorithmic_bytes": int(bytes_qkvo if dom == "sparse_attention" else
+                                          bytes_drift if dom == "drift_check" else bytes_score)})
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -268,6 +293,7 @@ def run_ours(args, ws, rank, local):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                    "l2": "3 rotating input sets (%.0f MB each) > 126 MB L2; no flush" % (3 * H * N * d * elem / 1e6),
                    "step": "drift_check(force) + score_blocks + select_topp + sparse_attention"},
+        "call_ms_score_select_attend": round(float(stage_ms[1:].sum()), 5),
         "pct_bf16_peak_call": round(100.0 * att_flops / (ms_step * 1e-3) / 1e12 / bf16_peak, 3),
         "kept_blocks_per_row": round(kept_pairs / (H * plan.nb), 3),
         "kept_density": round(kept_pairs / (H * plan.nb * plan.nb), 5),
@@ -281,20 +307,26 @@ def run_ours(args, ws, rank, local):
 
 # ------------------------------------------------------------------------- oracle
 
-def oracle_call_ms(w, Qb, Kb, Vb, mode, heads_sample):
-    """Time the oracle's drift + score + select + attention on a sample of heads; returns
-    (ms per call extrapolated to all heads, seconds spent, heads used)."""
+def oracle_call_ms(w, Qb, Kb, Vb, mode, heads_sample, min_seconds=0.0):
+    """Time the oracle's drift + score + select + attention head by head: the heads of
+    `heads_sample` first, then further heads in order (cycling) until `min_seconds` of CPU
+    work have passed. Returns (ms per call extrapolated to all heads, seconds spent, head
+    calls made)."""
     from oracle import bsa_oracle as O
     L = O.block_layout(w.T, w.H, w.W, w.text_tokens, w.block)
     t = time.perf_counter()
-    for h in heads_sample:
+    calls = 0
+    order = list(heads_sample)
+    while calls < len(order) or time.perf_counter() - t < min_seconds:
+        h = order[calls] if calls < len(order) else calls % w.heads
         Qh, Kh, Vh = O.bf16_to_f64(Qb[h]), O.bf16_to_f64(Kb[h]), O.bf16_to_f64(Vb[h])
         O.drift(Qh, Kh, Qh, Kh)
         S = O.score_head(Qh, Kh, L, mode).astype(np.float32)
         idx, cnt = O.select_topp(S, w.p[h], L)
         O.sparse_attention_head(Qh, Kh, Vh, idx, cnt, L)
+        calls += 1
     dt = time.perf_counter() - t
-    return dt / len(heads_sample) * w.heads * 1e3, dt, len(heads_sample)
+    return dt / calls * w.heads * 1e3, dt, calls
 
 
 def cpu_threads():
@@ -342,7 +374,9 @@ def main():
     ap.add_argument("--mode", default="meanpool", choices=["meanpool", "park"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-heads", type=int, default=3, help="heads in the bounded oracle sample")
+    ap.add_argument("--cpu-heads", type=int, default=1, help="heads the bounded oracle sample starts with")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU seconds the oracle sample runs for (whole heads, at least --cpu-heads)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (None if stale)")
     args = ap.parse_args()
@@ -372,10 +406,12 @@ def main():
             import torch
             Qb, Kb, Vb = (x.view(torch.int16).cpu().numpy().view(np.uint16) for x in sets[0])
             heads = list(range(min(args.cpu_heads, w.heads)))
-            ms, secs, nh = oracle_call_ms(w, Qb, Kb, Vb, "park" if args.mode == "park" else "meanpool", heads)
+            ms, secs, nh = oracle_call_ms(w, Qb, Kb, Vb, "park" if args.mode == "park" else "meanpool", heads,
+                                          args.cpu_seconds)
             line["cpu_baseline"] = {"value": round(ms, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                                    "sample": f"{nh} of {w.heads} heads, full drift+score+select+attention, "
-                                              f"{secs:.1f} s of CPU work, extrapolated to all heads"}
+                                    "sample": f"{nh} single-head calls (heads 0.. in order, cycling; {w.heads} heads "
+                                              f"per layer), full drift+score+select+attention, {secs:.1f} s of CPU "
+                                              f"work, mean per head x {w.heads}"}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
