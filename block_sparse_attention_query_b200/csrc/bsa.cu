@@ -9,6 +9,7 @@
 #include "bsa_common.cuh"
 #include "score.cuh"
 #include "park_tc.cuh"
+#include "meanpool_tc.cuh"
 #include "select.cuh"
 #include "drift.cuh"
 #include "attention.cuh"
@@ -81,10 +82,16 @@ size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(i
 // Score workspace: [pooled Q means | pooled K means: heads*nb*d fp32 each][block-slot table]
 size_t pooled_bytes(const Geom& g) { return align256((size_t)2 * g.heads * g.nb * g.d * sizeof(float)); }
 int park_nbp(const Geom& g) { return (g.nb + park::NT - 1) / park::NT * park::NT; }
-// PARK also keeps the three bf16 parts of the pooled keys: [heads][3][nbp][d]
+// Both scorers keep the three bf16 parts of the pooled keys, [heads][3][nbp][d]; the
+// mean-pooled one also those of the pooled queries, [heads][3][nbq][d] (nbq: nb rounded up to
+// a multiple of 128), then one float per score row (its softmax offset).
 size_t ksplit_bytes(const Geom& g) { return align256((size_t)g.heads * 3 * park_nbp(g) * g.d * 2); }
+int mp_nbq(const Geom& g) { return (g.nb + mp::BQ - 1) / mp::BQ * mp::BQ; }
+size_t qsplit_bytes(const Geom& g) { return align256((size_t)g.heads * 3 * mp_nbq(g) * g.d * 2); }
+size_t rowoff_bytes(const Geom& g) { return align256((size_t)g.heads * g.nb * sizeof(float)); }
 size_t score_ws_bytes(const Geom& g, int mode) {
-    return pooled_bytes(g) + perm_bytes(g) + (mode == BSA_SCORE_PARK ? ksplit_bytes(g) : 0);
+    return pooled_bytes(g) + perm_bytes(g) + ksplit_bytes(g) +
+           (mode == BSA_SCORE_MEANPOOL ? qsplit_bytes(g) + rowoff_bytes(g) : 0);
 }
 
 template <int D>
@@ -114,6 +121,41 @@ int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* 
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     const int grid = P.n_items < sms ? P.n_items : sms;
     park::park_tc_kernel<D><<<grid, park::kThreads, C::SMEM, st>>>(P);
+    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
+int sm_count();
+
+template <int D>
+int launch_meanpool(const Geom& g, const float* qbar, const float* kbar, const int* head_mask, float* scores,
+                    bsa_bf16* qsplit, bsa_bf16* ksplit, float* rowoff, cudaStream_t st) {
+    using C = mp::Cfg<D>;
+    const int nbq = mp_nbq(g), nbp = park_nbp(g);
+    const long long nq = (long long)g.heads * nbq * D, nk = (long long)g.heads * nbp * D;
+    park::split_kbar_kernel<D><<<(unsigned)((nq + 255) / 256), 256, 0, st>>>(g, qbar, nbq, qsplit);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    park::split_kbar_kernel<D><<<(unsigned)((nk + 255) / 256), 256, 0, st>>>(g, kbar, nbp, ksplit);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaFuncSetAttribute(mp::meanpool_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+        return BSA_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms <= 0) return BSA_ERR_CUDA;
+    mp::Params P;
+    P.g = g;
+    P.qsplit = qsplit;
+    P.ksplit = ksplit;
+    P.head_mask = head_mask;
+    P.scores = scores;
+    P.rowoff = rowoff;
+    P.nbq = nbq;
+    P.nbp = nbp;
+    P.n_items = g.heads * (nbq / mp::BQ);
+    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    const int grid = P.n_items < sms ? P.n_items : sms;
+    mp::meanpool_tc_kernel<D><<<grid, mp::kThreads, C::SMEM, st>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    mp::normalize_rows_kernel<<<g.heads * g.nb, 128, 0, st>>>(g, head_mask, rowoff, scores);
     return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 
@@ -229,11 +271,11 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
     else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
     if ((rc = launch_status()) != BSA_OK) return rc;
-    const float scale = 1.0f / std::sqrt((float)g.d);
-    if (prob->score_mode == BSA_SCORE_MEANPOOL) {
+    bsa_bf16* ksplit = reinterpret_cast<bsa_bf16*>(static_cast<uint8_t*>(ws) + pooled_bytes(g) + perm_bytes(g));
+    if (prob->score_mode == BSA_SCORE_MEANPOOL && (long long)g.heads * mp_nbq(g) / mp::BQ < sm_count()) {
+        // fewer 128-row items than SMs: the CUDA-core scorer with 8-32 rows per CTA
+        const float scale = 1.0f / std::sqrt((float)g.d);
         const int nbp = (g.nb + 3) & ~3;
-        // rows per CTA: as many as keep >= 2 CTAs per SM busy (fewer rows = more CTAs, but
-        // each CTA re-reads every pooled key of its head from L2); 16 at most past 1024 blocks
         int R = 32;
         if (g.nb > 1024) R = 16;
         while (R > 8 && (long long)((g.nb + R - 1) / R) * g.heads < 296) R >>= 1;
@@ -251,7 +293,12 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
 #undef BSA_MP
         return launch_status();
     }
-    bsa_bf16* ksplit = reinterpret_cast<bsa_bf16*>(static_cast<uint8_t*>(ws) + pooled_bytes(g) + perm_bytes(g));
+    if (prob->score_mode == BSA_SCORE_MEANPOOL) {
+        bsa_bf16* qsplit = reinterpret_cast<bsa_bf16*>(reinterpret_cast<uint8_t*>(ksplit) + ksplit_bytes(g));
+        float* rowoff = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(qsplit) + qsplit_bytes(g));
+        if (g.d == 128) return launch_meanpool<128>(g, qbar, kbar, head_mask, scores, qsplit, ksplit, rowoff, st);
+        return launch_meanpool<64>(g, qbar, kbar, head_mask, scores, qsplit, ksplit, rowoff, st);
+    }
     if (g.d == 128) return launch_park<128>(g, Q, kbar, perm, head_mask, scores, ksplit, st);
     return launch_park<64>(g, Q, kbar, perm, head_mask, scores, ksplit, st);
 }

@@ -1,11 +1,12 @@
-// Block pooling and the mean-pooled block scorer.
+// Block pooling and the CUDA-core mean-pooled block scorer.
 //
 // pool_kernel:  qbar[h][i] = mean of Q over the real tokens of block i (same for K).
 //   HBM-bound: every real row of Q and K is read exactly once, 16-byte loads, CD/8 lanes
 //   per 2*d-byte row, float32 accumulation, shared-memory tree reduction.
-// meanpool_score_kernel: S[h][i][j] = softmax_j(qbar_i . kbar_j / sqrt(d)) for 16 or 32
-//   query rows per CTA against every key block; register-blocked float32 dot products,
-//   row softmax in shared memory.
+// meanpool_score_kernel: S[h][i][j] = softmax_j(qbar_i . kbar_j / sqrt(d)) for 8, 16 or 32
+//   query rows per CTA against every key block; register-blocked float32 dot products, row
+//   softmax in shared memory. Used when the problem is too small to fill the SMs with the
+//   tensor-core scorer's 128-row items (meanpool_tc.cuh); same logits to float32 rounding.
 // (PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers,
 // Abstract: block retrieval from the averaged representations of query and key blocks.)
 #pragma once

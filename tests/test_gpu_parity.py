@@ -110,6 +110,27 @@ def test_scores_match_oracle(name, mode):
         assert np.allclose(S[h].sum(axis=1), 1.0, atol=1e-5)
 
 
+# Enough 128-row items (heads x query tiles >= SM count) that the mean-pooled scores take the
+# tensor-core path: several key tiles, a row count not a multiple of 4, text blocks.
+MANY_HEADS = {
+    "mh_d64_b64": dict(heads=150, d=64, T=5, H=32, W=52, text=0, B=64, p=0.9),
+    "mh_d128_b128_text": dict(heads=150, d=128, T=3, H=16, W=40, text=130, B=128, p=0.9),
+}
+
+
+@pytest.mark.parametrize("name", list(MANY_HEADS))
+def test_scores_tensor_core_path_match_oracle(name):
+    c = Case(**MANY_HEADS[name], mode="meanpool")
+    S = c.gpu_scores().cpu().numpy()
+    torch.cuda.synchronize()
+    _status_ok()
+    for h in range(0, c.heads, 7):
+        ref = c.oracle_scores(h)
+        err = np.abs(S[h] - ref)
+        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * ref), (h, float(err.max()))
+        assert np.allclose(S[h].sum(axis=1), 1.0, atol=1e-5)
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_select_on_oracle_scores_is_exact(name):
     # same float32 scores on both sides: only the cumulative-sum rounding may differ
