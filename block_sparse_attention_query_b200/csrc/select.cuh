@@ -140,17 +140,22 @@ __global__ void __launch_bounds__(kSelectThreads) select_topp_kernel(
 }
 
 
-// One warp per video query row with p < 1 (rows up to 1024 blocks). Lane l holds the keys
-// of blocks l, l+32, ...: key = ~float_bits(score), so an ascending key order is score
-// descending, and among equal keys the lower block index wins. The warp extracts the best
-// remaining block, adds its score to a float32 running sum (sequentially, in sorted order)
-// and stops once the sum reaches p -- usually after a handful of blocks. The kept list is
-// then merged with the forced text key blocks in the same order. A row that needs more than
+// One warp per video query row with p < 1 (rows up to 1024 blocks). Block j's key is
+// ~float_bits(score), so an ascending key order is score descending, and among equal keys the
+// lower block index wins; the row's keys sit in shared memory (lane l owns blocks l, l+32, ...),
+// which keeps registers, and so the number of resident warps, low. The warp extracts the best
+// remaining block, adds its score to a float32 running sum (sequentially, in sorted order) and
+// stops once the sum reaches p -- usually after a handful of blocks. The kept list is then
+// merged with the forced text key blocks in the same order. A row that needs more than
 // kWarpSelectCap extractions is marked cnt = -1 for the sorting kernel.
+constexpr int kWarpSelectMaxBlocks = 1024;
+
 template <int E>
 __global__ void __launch_bounds__(256) select_topp_warp_kernel(
     Geom g, const float* __restrict__ scores, const float* __restrict__ p,
     const int* __restrict__ head_mask, int* __restrict__ idx, int* __restrict__ cnt) {
+    static_assert(E * 32 <= kWarpSelectMaxBlocks, "row fits the key buffer");
+    __shared__ uint32_t key_s[8][E * 32];
     __shared__ int kept_s[8][kWarpSelectCap];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nb = g.nb;
@@ -162,33 +167,40 @@ __global__ void __launch_bounds__(256) select_topp_warp_kernel(
     const float pth = p[h];
     if (!(pth < 1.0f)) return;                                // keep-all rows: sorting kernel
     const float* srow = scores + (size_t)row * nb;
-    uint32_t key[E];
+    uint32_t* keys = key_s[warp];
+    float sc[E];
 #pragma unroll
     for (int m = 0; m < E; ++m) {
         const int j = lane + 32 * m;
-        uint32_t k = 0xFFFFFFFFu;
-        if (j < nb) {
-            const float sc = srow[j];
-            k = ~((sc > 0.f) ? __float_as_uint(sc) : 0u);    // not > 0 (0, -0, NaN) orders as 0
-        }
-        key[m] = k;
+        sc[m] = j < nb ? srow[j] : 0.f;                       // all loads in flight together
     }
     // lane-local best untaken block as (key << 32 | index); all ones when none is left (no
     // real block has that value: indices stay below 2^31)
     uint32_t taken = 0;                                     // bit m: block lane + 32m retired
+    unsigned long long mine = ~0ull;
 #pragma unroll
-    for (int m = 0; m < E; ++m)
-        if (lane + 32 * m >= nb) taken |= 1u << m;
+    for (int m = 0; m < E; ++m) {
+        const int j = lane + 32 * m;
+        if (j < nb) {
+            const uint32_t k = ~((sc[m] > 0.f) ? __float_as_uint(sc[m]) : 0u);   // not > 0 orders as 0
+            keys[j] = k;
+            const unsigned long long c = ((unsigned long long)k << 32) | (uint32_t)j;
+            if (c < mine) mine = c;
+        } else {
+            taken |= 1u << m;
+        }
+    }
+    __syncwarp();
     auto local_best = [&]() -> unsigned long long {
         unsigned long long b = ~0ull;
-#pragma unroll
         for (int m = 0; m < E; ++m) {
-            const unsigned long long c = ((unsigned long long)key[m] << 32) | (uint32_t)(lane + 32 * m);
-            if (!((taken >> m) & 1u) && c < b) b = c;
+            if ((taken >> m) & 1u) continue;
+            const int j = lane + 32 * m;
+            const unsigned long long c = ((unsigned long long)keys[j] << 32) | (uint32_t)j;
+            if (c < b) b = c;
         }
         return b;
     };
-    unsigned long long mine = local_best();
     float cum = 0.f;
     int n = 0;
     bool done = false;
@@ -218,10 +230,9 @@ __global__ void __launch_bounds__(256) select_topp_warp_kernel(
     __syncwarp();
     if (lane == 0) {
         // merge the kept prefix (already in key order) with the forced text blocks, taken
-        // in key order too (at most 64 text blocks reach this kernel)
+        // in key order too (at most 64 text blocks reach this kernel); keys from shared memory
         auto key_of = [&](int j) -> unsigned long long {
-            const float sc = srow[j];
-            return ((unsigned long long)(~((sc > 0.f) ? __float_as_uint(sc) : 0u)) << 32) | (uint32_t)j;
+            return ((unsigned long long)keys[j] << 32) | (uint32_t)j;
         };
         int* out = idx + (size_t)row * nb;
         unsigned long long used = 0;                     // bit t - nbv: text block placed
