@@ -106,8 +106,13 @@ int bsa_block_layout(const bsa_problem* prob, int* perm_host);
  *              their rows of `scores` are left untouched (the cached-mask case).
  *   scores     [heads, nb, nb] float32 out. Row (h, i) is a probability distribution over
  *              key blocks j (including text blocks); logits are scaled by 1/sqrt(d).
- *   ws         workspace of at least plan.score_workspace_bytes (pooled block means).
- * Mode is prob->score_mode. */
+ *   ws         workspace of at least plan.score_workspace_bytes: pooled block means, the
+ *              block-slot table, the bf16 three-way splits of the pooled keys (and, for the
+ *              mean-pooled mode, of the pooled queries and one offset per score row). Its
+ *              size depends on the mode, so plan with the mode that will run.
+ * Mode is prob->score_mode. Mean-pooled scores are float32-grade: float32 dot products on
+ * CUDA cores for problems too small to fill the GPU, otherwise tensor-core products of the
+ * bf16 splits; both agree with exact arithmetic to float32 rounding. */
 int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                      const int* head_mask, float* scores,
                      void* ws, size_t ws_bytes, bsa_stream_t stream);
