@@ -44,6 +44,24 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def max_over_ranks(x, ws, device):
+    """The slowest rank's value of a per-rank time (a collective over the process group when
+    there is more than one rank; every rank calls it at the same point)."""
+    if ws <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ms_per_step, ws):
+    """Whole-job ms per layer call: ws replicas each finish one layer call per step, so the job
+    completes ws calls in the slowest rank's step time."""
+    return ms_per_step / ws
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -187,10 +205,7 @@ def run_ours(args, ws, rank, local):
         for s in range(4):
             stage_ms[s] += e[s].elapsed_time(e[s + 1])
     stage_ms /= args.steps
-    if ws > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, ws, dev)
     ms_step = total_ms / args.steps
     st = bsa.bsa_device_status()
     if st != 0:
@@ -270,18 +285,15 @@ def run_ours(args, ws, rank, local):
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / e2e_steps
-        if ws > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(e2e_ms / ws, 4), "unit": UNIT,
+        e2e_ms = max_over_ranks(e2e_ms, ws, dev)
+        e2e = {"value": round(job_value(e2e_ms, ws), 4), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
 
     # drift (2) + block-slot table, pool, score (3) + select (warp pass unless every row is
     # sorted, sort pass) + block-slot table, attention (2) [+ text merge]
     sort_all = plan.nb > 1024 or plan.nb_text > 64
     launches_per_step = 2 + 3 + (1 if sort_all else 2) + 2 + (1 if plan.nb_text > 0 else 0)
-    value = ms_step / ws
+    value = job_value(ms_step, ws)
     line = {
         "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
