@@ -289,10 +289,19 @@ def run_ours(args, ws, rank, local):
         e2e = {"value": round(job_value(e2e_ms, ws), 4), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
 
-    # drift (2) + block-slot table, pool, score (3) + select (warp pass unless every row is
-    # sorted, sort pass) + block-slot table, attention (2) [+ text merge]
+    # drift (2) + score: block-slot table, pool, then the scorer [CUDA-core mean-pool: 1;
+    # tensor-core mean-pool (when heads x 128-row query tiles fill the SMs): 2 splits, scorer,
+    # row normalisation; PARK: split, scorer] + select (warp pass unless every row is sorted,
+    # sort pass) + block-slot table, attention [+ text merge]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    if args.mode == "park":
+        score_launches = 2 + 2
+    elif H * ((plan.nb + 127) // 128) < sms:
+        score_launches = 2 + 1
+    else:
+        score_launches = 2 + 4
     sort_all = plan.nb > 1024 or plan.nb_text > 64
-    launches_per_step = 2 + 3 + (1 if sort_all else 2) + 2 + (1 if plan.nb_text > 0 else 0)
+    launches_per_step = 2 + score_launches + (1 if sort_all else 2) + 2 + (1 if plan.nb_text > 0 else 0)
     value = job_value(ms_step, ws)
     line = {
         "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": ws,
