@@ -1,18 +1,22 @@
 """Benchmark of the block-sparse 3D attention hot path on B200.
 
-One step = one pass of the whole path over one layer of synthetic input resident in HBM:
+One step = one pass of the whole path over one attention layer of synthetic input resident in
+HBM:
     drift check (forced refresh: every head re-scores) -> block scores -> top-p select
     -> block-sparse attention
-on the Wan2.1-1.3B-shaped 480p layer (12 heads, d=128, 21x30x52 grid, 128-token blocks,
-p=0.9) unless --workload says otherwise. Three input sets rotate between steps (900 MB >
-126 MB L2), so no step finds its inputs in L2.
+on the HunyuanVideo-shaped 720p 5 s layer (24 heads, d=128, 33x45x80 grid + 256 text tokens,
+128-token blocks, p=0.9; the largest layer of the five workloads) unless --workload says
+otherwise. Its inputs (2.2 GB) are far larger than the 126 MB L2, so no step finds them in L2;
+smaller layers rotate three input sets.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--mode meanpool|park]
+                    [--workload NAME] [--mode meanpool|park] [--gather]
 
-Prints one JSON line. Multi-GPU (torchrun): each rank runs its own layer (replicas of the
-same shape, no collective on the data path); value = max-over-ranks step time divided by
-the calls all ranks made (ms per call, whole job).
+Prints one JSON line. Multi-GPU (torchrun, one rank per GPU): the layer's heads are split into
+N contiguous ranges and rank r runs the same C-ABI calls on heads [r*H/N, (r+1)*H/N). Every
+step of the path is per head, so the data path has no collective; --gather adds an NCCL
+all-gather of O (for a caller that wants every head's output on every GPU). value = the
+slowest rank's time per layer call (strong scaling: the layer is fixed and N GPUs share it).
 """
 from __future__ import annotations
 
@@ -33,6 +37,8 @@ sys.path.insert(0, ROOT)
 METRIC = "ms per sparse-attn call & % bf16 tensor peak (score+select+attend), 1 B200"
 UNIT = "ms"
 TAU = 0.05
+L2_BYTES = 126 * 2 ** 20
+DEFAULT_WORKLOAD = "hunyuan_720p"
 
 
 def _peaks():
@@ -42,6 +48,12 @@ def _peaks():
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def head_range(heads, ws, rank):
+    """Contiguous heads [h0, h1) of rank `rank` when `heads` are split over `ws` ranks (sizes
+    differ by at most one)."""
+    return rank * heads // ws, (rank + 1) * heads // ws
 
 
 def max_over_ranks(x, ws, device):
@@ -56,10 +68,14 @@ def max_over_ranks(x, ws, device):
     return float(t.item())
 
 
-def job_value(ms_per_step, ws):
-    """Whole-job ms per layer call: ws replicas each finish one layer call per step, so the job
-    completes ws calls in the slowest rank's step time."""
-    return ms_per_step / ws
+def sum_over_ranks(x, ws, device):
+    if ws <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 def _dist():
@@ -117,25 +133,34 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- ours
 
-def _profiled_traffic(kernel, workload):
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary, or None
-    when the kernel sources changed since that capture or the workload differs."""
-    if kernel != "sparse_attention":
-        return None
-    root = os.path.dirname(os.path.abspath(__file__))
-    prof = os.path.join(root, "profiles", f"sparse_attention_{workload}.md")
-    if not os.path.exists(prof):
-        return None
-    fields = {}
-    for line in open(prof):
-        k, sep, v = line.strip().partition(": ")
-        if sep and k in ("traffic_bytes_per_launch", "workload", "sources_sha256_16"):
-            fields[k] = v.strip()
+def _sources_hash(root):
     src = b"".join(open(os.path.join(root, "block_sparse_attention_query_b200", "csrc", f), "rb").read()
                    for f in ("attention.cuh", "bsa_common.cuh"))
-    if fields.get("workload") != workload or fields.get("sources_sha256_16") != hashlib.sha256(src).hexdigest()[:16]:
+    return hashlib.sha256(src).hexdigest()[:16]
+
+
+def _profiled_traffic(kernel, workload, root=None):
+    """DRAM bytes per launch of the attention kernel from the committed ncu figures
+    (profiles/sparse_attention_<workload>.json), or None when the kernel sources changed since
+    that capture or no capture exists for the workload."""
+    if kernel != "sparse_attention":
+        return None
+    root = root or os.path.dirname(os.path.abspath(__file__))
+    prof = os.path.join(root, "profiles", f"sparse_attention_{workload}.json")
+    if not os.path.exists(prof):
+        return None
+    with open(prof) as f:
+        fields = json.load(f)
+    if fields.get("workload") != workload or fields.get("sources_sha256_16") != _sources_hash(root):
         return None
     return int(fields["traffic_bytes_per_launch"])
+
+
+def _input_sets(w, h0, h1, n_sets, rank):
+    from block_sparse_attention_query_b200 import inputs
+    workers = max(1, min(os.cpu_count() or 1, 16, h1 - h0))
+    return [inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=s,
+                                head_range=(h0, h1), workers=workers) for s in range(n_sets)]
 
 
 def run_ours(args, ws, rank, local):
@@ -145,18 +170,23 @@ def run_ours(args, ws, rank, local):
     from block_sparse_attention_query_b200 import bsa, inputs
     from block_sparse_attention_query_b200.layer import SparseAttentionLayer
 
+    w = inputs.workload(args.workload)
+    h0, h1 = head_range(w.heads, ws, rank)
+    Hl = h1 - h0
+    B, d, N = w.block, w.d, w.tokens
+    elem = 2
+    local_set_bytes = 3 * Hl * N * d * elem
+    n_sets = 1 if local_set_bytes >= 4 * L2_BYTES else 3
+    host_sets = _input_sets(w, h0, h1, n_sets, rank)   # drawn before the first CUDA call
+
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = inputs.workload(args.workload)
     mode = bsa.BSA_SCORE_PARK if args.mode == "park" else bsa.BSA_SCORE_MEANPOOL
-    n_sets = 3
-    sets = []
-    for s in range(n_sets):
-        Qb, Kb, Vb = inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=s + 17 * rank)
-        sets.append(tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (Qb, Kb, Vb)))
-    layer = SparseAttentionLayer(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, p=list(w.p),
+    sets = [tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in hs) for hs in host_sets]
+    layer = SparseAttentionLayer(Hl, d, w.T, w.H, w.W, w.text_tokens, B, p=list(w.p[h0:h1]),
                                  tau=TAU, score_mode=mode, device=dev)
-    O = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device=dev)
+    O = torch.empty(Hl, N, d, dtype=torch.bfloat16, device=dev)
+    O_all = torch.empty(ws, Hl, N, d, dtype=torch.bfloat16, device=dev) if (args.gather and ws > 1) else None
     stream = torch.cuda.current_stream(dev)
     prob, plan = layer.prob, layer.plan
 
@@ -176,6 +206,8 @@ def run_ours(args, ws, rank, local):
         bsa.bsa_sparse_attention(prob, Q, K, V, layer.idx, layer.cnt, O, layer.ws_attn)
         if ev is not None:
             ev[4].record(stream)
+        if O_all is not None:
+            dist.all_gather_into_tensor(O_all.view(-1), O.view(-1))
 
     for k in range(args.warmup):
         step(k)
@@ -191,11 +223,13 @@ def run_ours(args, ws, rank, local):
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = bsa.bsa_launch_count()
     t0.record(stream)
     for k in range(args.steps):
         step(k, evs[k])
     t1.record(stream)
     torch.cuda.synchronize()
+    launches = bsa.bsa_launch_count() - launches0
     if ws > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -206,22 +240,25 @@ def run_ours(args, ws, rank, local):
             stage_ms[s] += e[s].elapsed_time(e[s + 1])
     stage_ms /= args.steps
     total_ms = max_over_ranks(total_ms, ws, dev)
+    stage_ms = np.array([max_over_ranks(x, ws, dev) for x in stage_ms])
     ms_step = total_ms / args.steps
     st = bsa.bsa_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timing")
 
-    # work accounting from the masks the last step produced
+    # work accounting from the masks the last step produced (all ranks' heads)
     cnt = layer.cnt.cpu().numpy().astype(np.int64)
-    kept_pairs = int(cnt.sum())
-    B, d, N, H = w.block, w.d, w.tokens, w.heads
+    kept_pairs = int(sum_over_ranks(int(cnt.sum()), ws, dev))
+    launches = int(sum_over_ranks(launches, ws, dev))
+    H = w.heads
     att_flops = kept_pairs * 4.0 * B * B * d
     dense_flops = 4.0 * N * N * d * H
-    elem = 2
     bytes_qkvo = 4.0 * H * N * d * elem
     bytes_drift = 6.0 * H * N * d * elem              # read Q,K,Qref,Kref; write Qref,Kref
     bytes_score = 2.0 * H * N * d * elem              # read Q,K once (pooling)
     hbm, bf16_peak, bf16_sus, peak_src = _peaks()
+    # per-GPU rates: each GPU does 1/ws of the work in the (slowest rank's) stage time
+    per_gpu = 1.0 / ws
 
     stages = {}
     names = ["drift_check", "score_blocks", "select_topp", "sparse_attention"]
@@ -231,36 +268,39 @@ def run_ours(args, ws, rank, local):
     stages["sparse_attention"].update({
         "tflops_actual": round(att_flops / att_s / 1e12, 2),
         "tflops_dense_equiv": round(dense_flops / att_s / 1e12, 2),
-        "frac_bf16_peak": round(att_flops / att_s / 1e12 / bf16_peak, 4),
+        "frac_bf16_peak": round(att_flops * per_gpu / att_s / 1e12 / bf16_peak, 4),
         "hbm_gbs_compulsory": round(bytes_qkvo / att_s / 1e9, 1),
-        "frac_hbm": round(bytes_qkvo / att_s / 1e9 / hbm, 4)})
+        "frac_hbm": round(bytes_qkvo * per_gpu / att_s / 1e9 / hbm, 4)})
     stages["drift_check"].update({"gbs": round(bytes_drift / (stage_ms[0] * 1e-3) / 1e9, 1),
-                                  "frac_hbm": round(bytes_drift / (stage_ms[0] * 1e-3) / 1e9 / hbm, 4)})
+                                  "frac_hbm": round(bytes_drift * per_gpu / (stage_ms[0] * 1e-3) / 1e9 / hbm, 4)})
     stages["score_blocks"].update({"gbs": round(bytes_score / (stage_ms[1] * 1e-3) / 1e9, 1),
-                                   "frac_hbm": round(bytes_score / (stage_ms[1] * 1e-3) / 1e9 / hbm, 4)})
+                                   "frac_hbm": round(bytes_score * per_gpu / (stage_ms[1] * 1e-3) / 1e9 / hbm, 4)})
 
-    # dominant kernel roofline
+    # dominant kernel roofline (per GPU)
     dom = names[int(np.argmax(stage_ms))]
     if dom == "sparse_attention":
         t_tensor = att_flops / (bf16_peak * 1e12)
         t_hbm = bytes_qkvo / (hbm * 1e9)
         if t_tensor >= t_hbm:
-            ach = att_flops / att_s / 1e12
+            ach = att_flops * per_gpu / att_s / 1e12
             roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": bf16_peak, "unit": "TFLOP/s",
                     "frac": round(ach / bf16_peak, 4)}
         else:
-            ach = bytes_qkvo / att_s / 1e9
+            ach = bytes_qkvo * per_gpu / att_s / 1e9
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(ach / hbm, 4)}
     else:
         b = bytes_drift if dom == "drift_check" else bytes_score
-        ach = b / (stage_ms[names.index(dom)] * 1e-3) / 1e9
+        ach = b * per_gpu / (stage_ms[names.index(dom)] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4)}
-    traffic = args.traffic if args.traffic is not None else _profiled_traffic(dom, w.name)
-    roof.update({"kernel": dom, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
+    traffic = args.traffic if args.traffic is not None else (_profiled_traffic(dom, w.name) if ws == 1 else None)
+    roof.update({"kernel": dom,
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
                  "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
-                 "algorithmic_bytes": int(bytes_qkvo if dom == "sparse_attention" else
-                                          bytes_drift if dom == "drift_check" else bytes_score)})
+                 "algorithmic_bytes": int((bytes_qkvo if dom == "sparse_attention" else
+                                           bytes_drift if dom == "drift_check" else bytes_score) * per_gpu)})
+    if dom == "sparse_attention":
+        roof["algorithmic_flops"] = int(att_flops * per_gpu)
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -270,84 +310,67 @@ def run_ours(args, ws, rank, local):
             hx.copy_(dx)
         hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
         Qd, Kd, Vd = (torch.empty_like(x) for x in sets[0])
-        e2e_steps = max(3, min(args.steps, 20))
-        for _ in range(2):
+
+        def e2e_step():
             Qd.copy_(hQ, non_blocking=True); Kd.copy_(hK, non_blocking=True); Vd.copy_(hV, non_blocking=True)
             layer.step(Qd, Kd, Vd, O, force_refresh=True)
             hO.copy_(O, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            e2e_step()
         torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(e2e_steps):
-            Qd.copy_(hQ, non_blocking=True); Kd.copy_(hK, non_blocking=True); Vd.copy_(hV, non_blocking=True)
-            layer.step(Qd, Kd, Vd, O, force_refresh=True)
-            hO.copy_(O, non_blocking=True)
+            e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / e2e_steps
-        e2e_ms = max_over_ranks(e2e_ms, ws, dev)
-        e2e = {"value": round(job_value(e2e_ms, ws), 4), "unit": UNIT,
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, ws, dev)
+        e2e = {"value": round(e2e_ms, 4), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
 
-    # drift (2) + score: block-slot table, pool, then the scorer [CUDA-core mean-pool: 1;
-    # tensor-core mean-pool (when heads x 128-row query tiles fill the SMs): 2 splits, scorer,
-    # row normalisation; PARK: split, scorer] + select (warp pass unless every row is sorted,
-    # sort pass) + block-slot table, attention [+ text merge]
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    if args.mode == "park":
-        score_launches = 2 + 2
-    elif H * ((plan.nb + 127) // 128) < sms:
-        score_launches = 2 + 1
-    else:
-        score_launches = 2 + 4
-    sort_all = plan.nb > 1024 or plan.nb_text > 64
-    launches_per_step = 2 + score_launches + (1 if sort_all else 2) + 2 + (1 if plan.nb_text > 0 else 0)
-    value = job_value(ms_step, ws)
     line = {
-        "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": ws,
+        "metric": METRIC, "value": round(ms_step, 5), "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded RFF-structured Q/K, Gaussian V; no model weights)",
         "config": {"workload": w.name, "heads": H, "d": d, "grid": [w.T, w.H, w.W],
                    "text_tokens": w.text_tokens, "tokens": N, "block": B, "blocks": plan.nb,
                    "top_p": sorted(set(float(x) for x in w.p)), "scorer": args.mode,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": "3 rotating input sets (%.0f MB each) > 126 MB L2; no flush" % (3 * H * N * d * elem / 1e6),
+                   "parallelism": (f"heads split over {ws} GPUs, {Hl} per GPU, no data-path collective"
+                                   + (", all-gather of O" if O_all is not None else "")) if ws > 1 else "single GPU",
+                   "l2": (f"{n_sets} rotating input sets of {local_set_bytes / 1e6:.0f} MB per GPU "
+                          f"(> 126 MB L2); no flush"),
                    "step": "drift_check(force) + score_blocks + select_topp + sparse_attention"},
         "call_ms_score_select_attend": round(float(stage_ms[1:].sum()), 5),
-        "pct_bf16_peak_call": round(100.0 * att_flops / (ms_step * 1e-3) / 1e12 / bf16_peak, 3),
+        "pct_bf16_peak_call": round(100.0 * att_flops * per_gpu / (ms_step * 1e-3) / 1e12 / bf16_peak, 3),
         "kept_blocks_per_row": round(kept_pairs / (H * plan.nb), 3),
         "kept_density": round(kept_pairs / (H * plan.nb * plan.nb), 5),
         "tflops_actual_call": round(att_flops / (ms_step * 1e-3) / 1e12, 2),
         "tflops_dense_equiv_call": round(dense_flops / (ms_step * 1e-3) / 1e12, 2),
         "stages": stages, "roofline": roof, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        "gpu_launches": launches, "gpu_launches_per_step": round(launches / args.steps / ws, 2),
+        "clocks": clocks,
     }
-    return line, (w, sets if rank == 0 else None)
+    return line, (w, host_sets[0] if (rank == 0 and ws == 1) else None)
 
 
 # ------------------------------------------------------------------------- oracle
 
-def oracle_call_ms(w, Qb, Kb, Vb, mode, heads_sample, min_seconds=0.0):
-    """Time the oracle's drift + score + select + attention head by head: the heads of
-    `heads_sample` first, then further heads in order (cycling) until `min_seconds` of CPU
-    work have passed. Returns (ms per call extrapolated to all heads, seconds spent, head
-    calls made)."""
+def oracle_head_ms(w, Qb, Kb, Vb, mode, h_local, h_global):
+    """One head's drift + score + select + attention through the oracle; returns ms."""
     from oracle import bsa_oracle as O
     L = O.block_layout(w.T, w.H, w.W, w.text_tokens, w.block)
     t = time.perf_counter()
-    calls = 0
-    order = list(heads_sample)
-    while calls < len(order) or time.perf_counter() - t < min_seconds:
-        h = order[calls] if calls < len(order) else calls % w.heads
-        Qh, Kh, Vh = O.bf16_to_f64(Qb[h]), O.bf16_to_f64(Kb[h]), O.bf16_to_f64(Vb[h])
-        O.drift(Qh, Kh, Qh, Kh)
-        S = O.score_head(Qh, Kh, L, mode).astype(np.float32)
-        idx, cnt = O.select_topp(S, w.p[h], L)
-        O.sparse_attention_head(Qh, Kh, Vh, idx, cnt, L)
-        calls += 1
-    dt = time.perf_counter() - t
-    return dt / calls * w.heads * 1e3, dt, calls
+    Qh, Kh, Vh = O.bf16_to_f64(Qb[h_local]), O.bf16_to_f64(Kb[h_local]), O.bf16_to_f64(Vb[h_local])
+    O.drift(Qh, Kh, Qh, Kh)
+    S = O.score_head(Qh, Kh, L, mode).astype(np.float32)
+    idx, cnt = O.select_topp(S, w.p[h_global], L)
+    O.sparse_attention_head(Qh, Kh, Vh, idx, cnt, L)
+    return (time.perf_counter() - t) * 1e3
 
 
 def cpu_threads():
@@ -361,27 +384,52 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
+def cpu_baseline(w, Qb, Kb, Vb, mode, seconds):
+    """The oracle timed on the host cores on a bounded sample: whole heads (0, 1, ... in
+    order) until `seconds` of CPU work have passed, at least one; mean per head x heads."""
+    t = time.perf_counter()
+    per = []
+    while not per or time.perf_counter() - t < seconds:
+        h = len(per) % Qb.shape[0]
+        per.append(oracle_head_ms(w, Qb, Kb, Vb, mode, h, h))
+    ms = float(np.mean(per)) * w.heads
+    return {"value": round(ms, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{len(per)} single-head calls (heads 0.. in order, cycling; {w.heads} heads per layer), "
+                      f"full drift+score+select+attention, {time.perf_counter() - t:.1f} s of CPU work, "
+                      f"mean per head x {w.heads}"}
+
+
 def run_reference(args):
+    """The oracle on the host cores, as it stands. Each step runs one head of the layer through
+    the whole path (the next head each step); value = mean per-head time x heads, the same
+    metric (ms per layer call) as the GPU arm."""
     from block_sparse_attention_query_b200 import inputs
     w = inputs.workload(args.workload)
-    Qb, Kb, Vb = inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=0)
+    n_heads = min(w.heads, args.warmup + args.steps)
+    Qb, Kb, Vb = inputs.generate_qkv(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=0,
+                                     head_range=(0, n_heads), workers=min(os.cpu_count() or 1, 16))
     mode = "park" if args.mode == "park" else "meanpool"
     per_step = []
+    t_all = time.perf_counter()
     for k in range(args.warmup + args.steps):
-        h = k % w.heads
-        ms, _, _ = oracle_call_ms(w, Qb, Kb, Vb, mode, [h])
+        h = k % n_heads
+        ms = oracle_head_ms(w, Qb, Kb, Vb, mode, h, h)
         if k >= args.warmup:
             per_step.append(ms)
-    v = float(np.mean(per_step))
+    ms_head = float(np.mean(per_step))
+    v = ms_head * w.heads
     cores = cpu_threads()
-    sample = f"1 of {w.heads} heads per step (full drift+score+select+attention of that head), extrapolated x{w.heads}"
+    sample = (f"{args.steps} timed steps, each one head of {w.heads} (heads cycling) through the whole path "
+              f"(drift+score+select+attention); value = mean per-head time x {w.heads}")
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_head, 3),
+        "step": "one head of the layer through the oracle", "heads_timed_per_step": 1,
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "scorer": mode, "parallelism": "single process (host cores)"},
         "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s_timed_and_warmup": round(time.perf_counter() - t_all, 1),
     }
 
 
@@ -444,16 +492,16 @@ def run_reuse(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="wan13b_480p")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--mode", default="meanpool", choices=["meanpool", "park"])
+    ap.add_argument("--gather", action="store_true", help="all-gather O over the ranks every step (N > 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-heads", type=int, default=1, help="heads the bounded oracle sample starts with")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="CPU seconds the oracle sample runs for (whole heads, at least --cpu-heads)")
+                    help="CPU seconds the oracle sample runs for (whole heads, at least one)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (None if stale)")
     ap.add_argument("--reuse", type=int, default=0,
@@ -461,6 +509,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank, local = _dist()
+    if args.gather and ws > 1:
+        from block_sparse_attention_query_b200 import inputs
+        if inputs.workload(args.workload).heads % ws:
+            raise SystemExit("--gather needs the heads to split evenly over the GPUs")
 
     if args.reuse > 0:
         from block_sparse_attention_query_b200 import build
@@ -485,18 +537,11 @@ def main():
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
-    line, (w, sets) = run_ours(args, ws, rank, local)
+    line, (w, host0) = run_ours(args, ws, rank, local)
     if rank == 0:
-        if not args.no_cpu_baseline:
-            import torch
-            Qb, Kb, Vb = (x.view(torch.int16).cpu().numpy().view(np.uint16) for x in sets[0])
-            heads = list(range(min(args.cpu_heads, w.heads)))
-            ms, secs, nh = oracle_call_ms(w, Qb, Kb, Vb, "park" if args.mode == "park" else "meanpool", heads,
-                                          args.cpu_seconds)
-            line["cpu_baseline"] = {"value": round(ms, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                                    "sample": f"{nh} single-head calls (heads 0.. in order, cycling; {w.heads} heads "
-                                              f"per layer), full drift+score+select+attention, {secs:.1f} s of CPU "
-                                              f"work, mean per head x {w.heads}"}
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, host0[0], host0[1], host0[2],
+                                                "park" if args.mode == "park" else "meanpool", args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

@@ -73,6 +73,7 @@ EXPORTS = {
     "bsa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bsa_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_version": (ctypes.c_char_p, []),
+    "bsa_launch_count": (ctypes.c_ulonglong, []),
 }
 
 
@@ -173,3 +174,7 @@ def bsa_device_status(stream=None) -> int:
 
 def bsa_version() -> str:
     return lib.bsa_version().decode()
+
+
+def bsa_launch_count() -> int:
+    return int(lib.bsa_launch_count())

@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
+    const unsigned epoch = timeout_epoch();   // waits give up early only on a newer timeout
     const int nb = g.nb;
 
     if (threadIdx.x == 0) {
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             const RowToks<D, BQ> tq = load_tokens<D, BQ>(P, it.i, lt);
             RowToks<D, BK> tk = load_tokens<D, BK>(P, kept_block(it, 0), lt);
             int kb_ahead = it.n > 1 ? kept_block(it, 1) : 0;
-            if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1);
+            if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch);
             if (!ok) break;
             gather_tile<D, BQ>(tq, P.Q + head_off, sQ + qb * C::Q_BYTES, lt);
             cp_async_arrive_noinc(&q_full[qb]);
@@ -360,11 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                     tk = load_tokens<D, BK>(P, kb_ahead, lt);
                     if (j + 2 < it.n) kb_ahead = kept_block(it, j + 2);
                 }
-                if (gblk >= NK) ok = mbar_wait(&k_empty[ks], ((gblk / NK) - 1) & 1);
+                if (gblk >= NK) ok = mbar_wait(&k_empty[ks], ((gblk / NK) - 1) & 1, epoch);
                 if (!ok) break;
                 gather_tile<D, BK>(cur, P.K + head_off, sK + ks * C::KV_BYTES, lt);
                 cp_async_arrive_noinc(&k_full[ks]);
-                if (gblk >= NV) ok = mbar_wait(&v_empty[vs], ((gblk / NV) - 1) & 1);
+                if (gblk >= NV) ok = mbar_wait(&v_empty[vs], ((gblk / NV) - 1) & 1, epoch);
                 if (!ok) break;
                 gather_tile<D, BK>(cur, P.V + head_off, sV + vs * C::KV_BYTES, lt);
                 cp_async_arrive_noinc(&v_full[vs]);
@@ -380,9 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             // read from S buffer gb&1 (key k at column k/2: 8 columns per 16 keys).
             auto issue_pv = [&](int gb, int j, int kitem, bool last) -> bool {
                 const int ob = kitem & 1;
-                if (j == 0 && kitem >= 2 && !mbar_wait(&o_free[ob], ((kitem >> 1) - 1) & 1)) return false;
-                if (!mbar_wait(&p_full[gb & 1], (gb >> 1) & 1)) return false;
-                if (!mbar_wait(&v_full[gb % NV], (gb / NV) & 1)) return false;
+                if (j == 0 && kitem >= 2 && !mbar_wait(&o_free[ob], ((kitem >> 1) - 1) & 1, epoch)) return false;
+                if (!mbar_wait(&p_full[gb & 1], (gb >> 1) & 1, epoch)) return false;
+                if (!mbar_wait(&v_full[gb % NV], (gb / NV) & 1, epoch)) return false;
                 tc_fence_after();
                 const uint32_t vbase = sV + (gb % NV) * C::KV_BYTES;
                 const uint32_t pcol = tmem + C::TMEM_S + (gb & 1) * BK;
@@ -405,11 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 const Item it = decode_item(P, item);
                 if (it.n <= 0) continue;
                 const int qb = k & 1;
-                ok = mbar_wait(&q_full[qb], (k >> 1) & 1);
+                ok = mbar_wait(&q_full[qb], (k >> 1) & 1, epoch);
                 for (int j = 0; j < it.n && ok; ++j, ++gblk) {
                     const int ks = gblk % NK, sb = gblk & 1;
-                    ok = mbar_wait(&k_full[ks], (gblk / NK) & 1);
-                    if (ok && gblk >= 2) ok = mbar_wait(&s_free[sb], ((gblk >> 1) - 1) & 1);
+                    ok = mbar_wait(&k_full[ks], (gblk / NK) & 1, epoch);
+                    if (ok && gblk >= 2) ok = mbar_wait(&s_free[sb], ((gblk >> 1) - 1) & 1, epoch);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t qbase = sQ + qb * C::Q_BYTES;
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             if (ok && prev_g >= 0) ok = issue_pv(prev_g, prev_j, prev_k, prev_last);
             // every MMA issued by this thread has completed once fin_bar flips
             tc_commit(fin_bar);
-            mbar_wait(fin_bar, 0);
+            mbar_drain(fin_bar, 0);
         }
         __syncwarp();
     } else if (warp < kEpiWarp0) {
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 const int g_cur = gblk + j;              // stream index of this block
                 const int kcount = block_count(g, kb);
                 if (j + 2 < it.n) kb = kept_block(it, j + 2);   // prefetch for the next block
-                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[grp], (g_cur >> 1) & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[grp], (g_cur >> 1) & 1, epoch));
                 if (!ok) break;
                 tc_fence_after();
                 // pass 1: max of the row's raw scores (padding keys excluded)
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 // its predecessor's entry, which keeps the two groups' entries in step.
                 float mprev = -INFINITY;
                 if (g_cur >= 1) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&m_ready[grp ^ 1], ((g_cur - 1) >> 1) & 1));
+                    ok = __all_sync(0xffffffffu, mbar_wait(&m_ready[grp ^ 1], ((g_cur - 1) >> 1) & 1, epoch));
                     if (!ok) break;
                     mprev = mch[(grp ^ 1) * BQ + r];
                 }
@@ -538,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 // issued after the PV two blocks back completed, and PV of this block waits
                 // for p_full), so a parity wait is exact even though most blocks skip it.
                 if (j >= 1 && __any_sync(0xffffffffu, m != mprev)) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (g_cur - 1) & 1));
+                    ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (g_cur - 1) & 1, epoch));
                     if (!ok) break;
                     tc_fence_after();
                     const float alpha = ex2(mprev - m);   // 1 for rows that kept their max
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             gblk += it.n;
             // hand this group's reference max and row sum to the epilogue; O buffer ob (and
             // its slots) must have been released by the epilogue of the item two back
-            if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((k >> 1) - 1) & 1));
+            if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((k >> 1) - 1) & 1, epoch));
             if (!ok) break;
             ml[(ob * 4 + 2 * grp) * BQ + r] = mref;
             ml[(ob * 4 + 2 * grp + 1) * BQ + r] = l;
@@ -596,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 }
             } else {
                 const int ob = k & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (k >> 1) & 1));
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ml_ready[ob], (k >> 1) & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (k >> 1) & 1, epoch));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ml_ready[ob], (k >> 1) & 1, epoch));
                 if (!ok) break;
                 tc_fence_after();
                 // O is relative to the reference of the item's last block, the larger of the two

@@ -1,6 +1,7 @@
 // libbsa host side: argument validation, planning and kernel launches behind the C ABI of
 // include/bsa.h. Single translation unit so that the device error word is shared by every
 // kernel of the library.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -77,6 +78,15 @@ int make_geom(const bsa_problem* prob, Geom* g) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Kernels this library has launched in this process (every launch is followed by exactly one
+// launch_status() call, which counts it).
+std::atomic<unsigned long long> g_launch_count{0};
+
+int launch_status() {
+    g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
 size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(int)); }
 
 // Score workspace: [pooled Q means | pooled K means: heads*nb*d fp32 each][block-slot table]
@@ -101,7 +111,7 @@ int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* 
     const int nbp = park_nbp(g);
     const long long n = (long long)g.heads * nbp * D;
     park::split_kbar_kernel<D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(g, kbar, nbp, ksplit);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
     if (cudaFuncSetAttribute(park::park_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
         return BSA_ERR_CUDA;
@@ -121,7 +131,7 @@ int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* 
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     const int grid = P.n_items < sms ? P.n_items : sms;
     park::park_tc_kernel<D><<<grid, park::kThreads, C::SMEM, st>>>(P);
-    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+    return launch_status();
 }
 
 int sm_count();
@@ -133,9 +143,9 @@ int launch_meanpool(const Geom& g, const float* qbar, const float* kbar, const i
     const int nbq = mp_nbq(g), nbp = park_nbp(g);
     const long long nq = (long long)g.heads * nbq * D, nk = (long long)g.heads * nbp * D;
     park::split_kbar_kernel<D><<<(unsigned)((nq + 255) / 256), 256, 0, st>>>(g, qbar, nbq, qsplit);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
     park::split_kbar_kernel<D><<<(unsigned)((nk + 255) / 256), 256, 0, st>>>(g, kbar, nbp, ksplit);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
     if (cudaFuncSetAttribute(mp::meanpool_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
         return BSA_ERR_CUDA;
@@ -154,9 +164,9 @@ int launch_meanpool(const Geom& g, const float* qbar, const float* kbar, const i
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     const int grid = P.n_items < sms ? P.n_items : sms;
     mp::meanpool_tc_kernel<D><<<grid, mp::kThreads, C::SMEM, st>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
     mp::normalize_rows_kernel<<<g.heads * g.nb, 128, 0, st>>>(g, head_mask, rowoff, scores);
-    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+    return launch_status();
 }
 
 int drift_chunks(const Geom& g) {
@@ -185,9 +195,6 @@ int sm_count() {
     return n;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
-
-int launch_status() { return cuda_status(cudaGetLastError()); }
 
 template <int D, int BK>
 int launch_attention(const attn::Params& P, cudaStream_t st) {
@@ -496,6 +503,8 @@ const char* bsa_error_string(int status) {
     }
 }
 
-const char* bsa_version(void) { return "bsa 0.1.0 sm_100a"; }
+const char* bsa_version(void) { return "bsa 0.2.0 sm_100a"; }
+
+unsigned long long bsa_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 
 }  // extern "C"

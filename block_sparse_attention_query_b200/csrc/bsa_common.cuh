@@ -66,14 +66,31 @@ __host__ __device__ inline int block_count(const Geom& g, int i) {
 
 // ------------------------------------------------------------------- error word
 
-// Device error word of this library (one per device): 0 = ok, else a BSA_ERR_* code.
+// Device error word of this library (one per device): 0 = ok, else the BSA_ERR_* code of the
+// first device-side problem. Sticky: it keeps that first code until bsa_device_status reads
+// and clears it. No kernel reads it, so a word left set by an earlier call changes nothing
+// in later calls.
 __device__ int g_error_word;
 
+// Number of bounded waits that ran out on this device, ever. A kernel reads it once at entry;
+// its waits give up early when it has moved since (another wait of the same launch, or of a
+// launch running beside it, ran out), so the roles of a CTA wind down together instead of
+// each waiting out its own limit. Errors other than a timeout do not move it.
+__device__ unsigned int g_timeouts;
+
 __device__ inline void raise_error(int code) { atomicCAS(&g_error_word, 0, code); }
-__device__ inline bool error_raised() { return *(volatile int*)&g_error_word != 0; }
+__device__ inline void raise_timeout() {
+    raise_error(BSA_ERR_TIMEOUT);
+    atomicAdd(&g_timeouts, 1u);
+}
+__device__ inline unsigned timeout_epoch() { return *(volatile unsigned*)&g_timeouts; }
+__device__ inline bool timed_out_since(unsigned epoch) { return *(volatile unsigned*)&g_timeouts != epoch; }
 
 // About 2 s at the highest SM clock: any wait longer than this is treated as a hang.
-constexpr long long kWaitLimitCycles = 4000000000LL;
+#ifndef BSA_WAIT_LIMIT_CYCLES
+#define BSA_WAIT_LIMIT_CYCLES 4000000000LL
+#endif
+constexpr long long kWaitLimitCycles = BSA_WAIT_LIMIT_CYCLES;
 
 // --------------------------------------------------------------------- PTX: misc
 
@@ -119,36 +136,26 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Non-blocking: has the phase with the given parity completed?
-__device__ inline bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-// Bounded spin on a phase that is expected to complete within a few hundred cycles (two
-// warps meeting); no suspension, so the wake-up is immediate.
-__device__ inline bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete. Gives up (returning false) after
+// kWaitLimitCycles, raising BSA_ERR_TIMEOUT, or as soon as a wait elsewhere has run out since
+// the kernel read `epoch` (timeout_epoch() at entry).
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned epoch) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_test(bar, parity)) {
-        if (error_raised()) return false;
-        if (clock64() - t0 > kWaitLimitCycles) { raise_error(BSA_ERR_TIMEOUT); return false; }
+    while (!mbar_try_wait(bar, parity)) {
+        if (timed_out_since(epoch)) return false;
+        if (clock64() - t0 > kWaitLimitCycles) { raise_timeout(); return false; }
     }
     return true;
 }
 
-// Wait for the phase with the given parity to complete. Gives up (raising
-// BSA_ERR_TIMEOUT) after kWaitLimitCycles or as soon as another thread raised an error.
-__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Teardown wait: for work already issued to the hardware (tensor-core operations, copies),
+// which completes whatever else went wrong. Stops only at the cycle limit.
+__device__ inline bool mbar_drain(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (error_raised()) return false;
-        if (clock64() - t0 > kWaitLimitCycles) { raise_error(BSA_ERR_TIMEOUT); return false; }
+        if (clock64() - t0 > kWaitLimitCycles) { raise_timeout(); return false; }
     }
     return true;
 }

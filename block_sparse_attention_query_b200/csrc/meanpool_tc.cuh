@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
+    const unsigned epoch = timeout_epoch();   // waits give up early only on a newer timeout
     const int nb = g.nb;
     const int ntiles = P.nbp / NT;
     const int qtiles = P.nbq / BQ;
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
         for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
             if (skip_item(item)) continue;
             const int h = item / qtiles, qt = item - h * qtiles;
-            if (k >= 1) ok = mbar_wait(q_empty, (k - 1) & 1);
+            if (k >= 1) ok = mbar_wait(q_empty, (k - 1) & 1, epoch);
             if (!ok) break;
             const bsa_bf16* qh = P.qsplit + (size_t)h * 3 * P.nbq * D;
 #pragma unroll
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             const bsa_bf16* kh = P.ksplit + (size_t)h * 3 * P.nbp * D;
             for (int t = 0; t < ntiles && ok; ++t, ++gt) {
                 const int s = gt % NS;
-                if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1);
+                if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1, epoch);
                 if (!ok) break;
 #pragma unroll
                 for (int sp = 0; sp < 3; ++sp) {
@@ -172,11 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             int gt = 0, k = 0;
             for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
                 if (skip_item(item)) continue;
-                ok = mbar_wait(q_full, k & 1);
+                ok = mbar_wait(q_full, k & 1, epoch);
                 for (int t = 0; t < ntiles && ok; ++t, ++gt) {
                     const int s = gt % NS, lb = gt & 1;
-                    ok = mbar_wait(&k_full[s], (gt / NS) & 1);
-                    if (ok && gt >= 2) ok = mbar_wait(&l_free[lb], ((gt >> 1) - 1) & 1);
+                    ok = mbar_wait(&k_full[s], (gt / NS) & 1, epoch);
+                    if (ok && gt >= 2) ok = mbar_wait(&l_free[lb], ((gt >> 1) - 1) & 1, epoch);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
                 ++k;
             }
             tc_commit(fin_bar);
-            mbar_wait(fin_bar, 0);
+            mbar_drain(fin_bar, 0);
         }
         __syncwarp();
     } else {
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             const int row0 = qt * BQ + warp * 32;           // the warp's first query block
             for (int t = 0; t < ntiles && ok; ++t, ++gt) {
                 const int lb = gt & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&l_full[lb], (gt >> 1) & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait(&l_full[lb], (gt >> 1) & 1, epoch));
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t v0[32], v1[32];

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
+    const unsigned epoch = timeout_epoch();   // waits give up early only on a newer timeout
     const int nb = g.nb;
     const int ntiles = P.nbp / NT;
 
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
             if (skip_item(item)) continue;
             const int h = item / nb, i = item - h * nb;
             const int qb = k & 1;
-            if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1);
+            if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch);
             if (!ok) break;
             const bsa_bf16* Qh = P.Q + (size_t)h * g.N * D;
             const int* slot = P.perm + i * g.B;
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
             for (int t2 = 0; t2 < 2 * ntiles && ok; ++t2, ++gt) {
                 const int t = t2 % ntiles;                   // pass A tiles, then pass B tiles
                 const int s = gt % NS;
-                if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1);
+                if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1, epoch);
                 if (!ok) break;
 #pragma unroll
                 for (int sp = 0; sp < 3; ++sp) {
@@ -196,11 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
             for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
                 if (skip_item(item)) continue;
                 const int qb = k & 1;
-                ok = mbar_wait(&q_full[qb], (k >> 1) & 1);
+                ok = mbar_wait(&q_full[qb], (k >> 1) & 1, epoch);
                 for (int t2 = 0; t2 < 2 * ntiles && ok; ++t2, ++gt) {
                     const int s = gt % NS, lb = gt & 1;
-                    ok = mbar_wait(&k_full[s], (gt / NS) & 1);
-                    if (ok && gt >= 2) ok = mbar_wait(&l_free[lb], ((gt >> 1) - 1) & 1);
+                    ok = mbar_wait(&k_full[s], (gt / NS) & 1, epoch);
+                    if (ok && gt >= 2) ok = mbar_wait(&l_free[lb], ((gt >> 1) - 1) & 1, epoch);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t qbase = sQ + qb * C::Q_BYTES;
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
                 ++k;
             }
             tc_commit(fin_bar);
-            mbar_wait(fin_bar, 0);
+            mbar_drain(fin_bar, 0);
         }
         __syncwarp();
     } else {
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
             for (int t2 = 0; t2 < 2 * ntiles && ok; ++t2, ++gt) {
                 const int t = t2 % ntiles, lb = gt & 1;
                 const bool pass_b = t2 >= ntiles;
-                ok = __all_sync(0xffffffffu, mbar_wait(&l_full[lb], (gt >> 1) & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait(&l_full[lb], (gt >> 1) & 1, epoch));
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t v0[32], v1[32];
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
                 cp[colbase + 1] = p[1];
                 // the four warps meet; threads 0..NT-1 finish their column
                 mbar_arrive(col_bar);
-                ok = __all_sync(0xffffffffu, mbar_wait(col_bar, col_phase & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait(col_bar, col_phase & 1, epoch));
                 ++col_phase;
                 if (!ok) break;
                 if (r < NT && jbase + r < nb) {

@@ -8,8 +8,10 @@ Recipe (the pages give no input distribution; these stand in for Wan2.1 / Hunyua
 activations, which need trained weights we do not have):
 
 * video tokens sit on a 3D grid (t, y, x) in raster order, x fastest;
-* per head h, in this order: omega_h ~ N(0, (1/8)^2) of shape [d, 3] (radians per grid
-  unit), b_h ~ U[0, 2*pi)^d, then Q noise, K noise, V;
+* head h draws from its own stream, PCG64 seeded by SeedSequence(seed, spawn_key=(h,)), so
+  any range of heads can be drawn alone (one GPU's share of the heads, or heads in parallel);
+  in this order: omega_h ~ N(0, (1/8)^2) of shape [d, 3] (radians per grid unit),
+  b_h ~ U[0, 2*pi)^d, then Q noise, K noise, V;
 * RFF(t, y, x)_c = sqrt(2) * cos(omega_c . (t, y, x) + b_c)  (unit variance per channel);
 * Q = 0.5 * N(0,1) + 2.0 * RFF,  K = 0.5 * N(0,1) + 2.0 * RFF (same RFF, fresh noise),
   V ~ N(0,1);
@@ -69,45 +71,65 @@ def _coords(T: int, H: int, W: int) -> np.ndarray:
     return np.stack([t.ravel(), y.ravel(), x.ravel()], axis=1).astype(np.float64)
 
 
-def generate_qkv(heads: int, d: int, T: int, H: int, W: int, text_tokens: int = 0,
-                 seed: int = 0, state: bool = False):
-    """Draw Q, K, V for one layer.
+def _head_rng(seed: int, h: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(h,))))
 
-    Returns (Q, K, V) as uint16 bf16 bits [heads, tokens, d]. With ``state=True`` also
-    returns the float32 pre-rounding Q and K (the random-walk state of the reuse run).
-    """
-    rng = np.random.Generator(np.random.PCG64(seed))
+
+def _generate_head(args):
+    """Q, K, V bits (and the float32 pre-rounding Q, K) of head h."""
+    h, d, T, H, W, text_tokens, seed = args
+    rng = _head_rng(seed, h)
     nv = T * H * W
     n = nv + text_tokens
     xyz = _coords(T, H, W)
-    Q = np.empty((heads, n, d), np.uint16)
-    K = np.empty((heads, n, d), np.uint16)
-    V = np.empty((heads, n, d), np.uint16)
-    Qs = np.empty((heads, n, d), np.float32) if state else None
-    Ks = np.empty((heads, n, d), np.float32) if state else None
-    for h in range(heads):
-        omega = rng.normal(0.0, 1.0 / 8.0, size=(d, 3))
-        b = rng.uniform(0.0, 2.0 * np.pi, size=d)
-        rff = (np.sqrt(2.0) * np.cos(xyz @ omega.T + b)).astype(np.float32)
-        qn = rng.standard_normal((n, d), dtype=np.float32)
-        kn = rng.standard_normal((n, d), dtype=np.float32)
-        vn = rng.standard_normal((n, d), dtype=np.float32)
-        q = qn * np.float32(0.5)
-        k = kn * np.float32(0.5)
-        q[:nv] += np.float32(2.0) * rff
-        k[:nv] += np.float32(2.0) * rff
-        # text tokens: plain N(0,1), no 3D structure
-        q[nv:] = qn[nv:]
-        k[nv:] = kn[nv:]
-        Q[h] = f32_to_bf16_bits(q)
-        K[h] = f32_to_bf16_bits(k)
-        V[h] = f32_to_bf16_bits(vn)
+    omega = rng.normal(0.0, 1.0 / 8.0, size=(d, 3))
+    b = rng.uniform(0.0, 2.0 * np.pi, size=d)
+    rff = (np.sqrt(2.0) * np.cos(xyz @ omega.T + b)).astype(np.float32)
+    qn = rng.standard_normal((n, d), dtype=np.float32)
+    kn = rng.standard_normal((n, d), dtype=np.float32)
+    vn = rng.standard_normal((n, d), dtype=np.float32)
+    q = qn * np.float32(0.5)
+    k = kn * np.float32(0.5)
+    q[:nv] += np.float32(2.0) * rff
+    k[:nv] += np.float32(2.0) * rff
+    # text tokens: plain N(0,1), no 3D structure
+    q[nv:] = qn[nv:]
+    k[nv:] = kn[nv:]
+    return f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(vn), q, k
+
+
+def generate_qkv(heads: int, d: int, T: int, H: int, W: int, text_tokens: int = 0,
+                 seed: int = 0, state: bool = False, head_range=None, workers: int = 1):
+    """Draw Q, K, V for one layer, or for the heads [h0, h1) of `head_range` only.
+
+    Returns (Q, K, V) as uint16 bf16 bits [h1 - h0, tokens, d]. With ``state=True`` also
+    returns the float32 pre-rounding Q and K (the random-walk state of the reuse run).
+    ``workers`` > 1 draws heads in that many spawned processes (the result is the same).
+    """
+    h0, h1 = (0, heads) if head_range is None else head_range
+    if not 0 <= h0 <= h1 <= heads:
+        raise ValueError("head range outside the layer")
+    jobs = [(h, d, T, H, W, text_tokens, seed) for h in range(h0, h1)]
+    if workers > 1 and len(jobs) > 1:
+        import concurrent.futures
+        import multiprocessing
+        with concurrent.futures.ProcessPoolExecutor(
+                max_workers=min(workers, len(jobs)), mp_context=multiprocessing.get_context("spawn")) as ex:
+            per_head = list(ex.map(_generate_head, jobs))
+    else:
+        per_head = [_generate_head(j) for j in jobs]
+    n = T * H * W + text_tokens
+    out = [np.empty((h1 - h0, n, d), np.uint16) for _ in range(3)]
+    st = [np.empty((h1 - h0, n, d), np.float32) for _ in range(2)] if state else None
+    for i, r in enumerate(per_head):
+        for a in range(3):
+            out[a][i] = r[a]
         if state:
-            Qs[h] = q
-            Ks[h] = k
+            st[0][i] = r[3]
+            st[1][i] = r[4]
     if state:
-        return Q, K, V, Qs, Ks
-    return Q, K, V
+        return out[0], out[1], out[2], st[0], st[1]
+    return out[0], out[1], out[2]
 
 
 def draw_top_p(heads: int, seed: int = 0) -> np.ndarray:

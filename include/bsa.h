@@ -34,6 +34,11 @@
  *     and returns a status code. Argument errors are detected on the host before anything is
  *     launched; nothing is written then. Device-side problems (a bounded wait that ran out, an
  *     out-of-range kept-block index) set a device error word read by bsa_device_status.
+ *     The word is sticky: it keeps the FIRST problem's code until bsa_device_status reads and
+ *     clears it, so read it after any sequence of calls whose results matter. No kernel reads
+ *     the word: later calls run normally whether or not it is set. A bad kept-block index
+ *     or count only spoils its own query block's output; a wait that ran out (about 2 s; a
+ *     hang) ends that launch early, and every output of that call is then unspecified.
  *   - Thread safety: calls only read their arguments; concurrent calls on different streams
  *     are safe as long as their output buffers and workspaces do not overlap.
  */
@@ -191,8 +196,13 @@ int bsa_device_status(bsa_stream_t stream);
 /* Static description of a status code (never NULL). */
 const char* bsa_error_string(int status);
 
-/* Library version, e.g. "bsa 0.1.0 sm_100a". */
+/* Library version, e.g. "bsa 0.2.0 sm_100a". */
 const char* bsa_version(void);
+
+/* Number of kernels this library has launched in this process so far (all devices, all
+ * streams; host counter, no CUDA call). A caller that wants the launches of a stretch of
+ * calls takes the difference of two readings. */
+unsigned long long bsa_launch_count(void);
 
 #ifdef __cplusplus
 }

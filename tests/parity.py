@@ -1,15 +1,46 @@
-"""Helpers for GPU-vs-oracle parity: device transfer and the kept-list comparison rule.
+"""Helpers for GPU-vs-oracle parity: device transfer, the score error bound and the kept-list
+comparison rule.
 
-Kept-list rule (top-p lists, per row):
-  * bit-exact lists pass;
-  * a different cut length passes when the oracle's float32 cumulative mass at the
-    boundary lies within WINDOW (1e-5) of p — the prefix must still be identical;
-  * position-wise substitutions pass only between blocks whose oracle scores agree within
-    the scorer's own float32 error (TIE_REL relative): the two scores are then not
-    distinguishable by the kernel's arithmetic, so either order is correct.
-Anything else is a true mismatch; the gate is zero true mismatches.
+Score error bound (one model, used both as the score tolerance and for near-ties in the
+kept lists). A block score is a softmax of logits x_j over key blocks. A float32 kernel
+computes x_j with an absolute error of at most u * E_j (u = 2^-24, E_j below); the
+normaliser then moves by at most the softmax-weighted mean of those errors, and the
+exponentials, the sum of nb terms and the division add at most u * K_norm relative. To first
+order the computed score S~_j satisfies
+
+    |S~_j - S_j| <= S_j * u * (E_j + sum_j' S_j' E_j' + K_norm)
+
+With s = 1/sqrt(d):
+
+  mean-pooled  x_ij = s * qbar_i . kbar_j, where qbar, kbar are float32 block means:
+      E_ij = K_DOT  * s * sum_c |qbar_ic| |kbar_jc|                      (the d-term dot product)
+           + K_POOL * s * sum_c (mean|Q|_ic |kbar_jc| + |qbar_ic| mean|K|_jc)   (the block sums)
+  PARK         x_qj = s * q . kbar_j per real query q, then averaged over the block's queries:
+      E_qj = K_DOT * s * sum_c |q_c| |kbar_jc| + K_POOL * s * sum_c |q_c| mean|K|_jc
+      |P~_ij - P_ij| <= mean_q p_qj u (E_qj + sum_j' p_qj' E_qj') + P_ij u K_norm
+
+Each E term is u times the sum of the magnitudes that the float32 sums round, times four
+(K_DOT = K_POOL = 4): the rounding errors of a sum partly cancel in any summation order, and
+single float32 logits of these inputs were seen up to 3.8 times that magnitude sum off (the
+worst case, n times, never comes near). K_norm = 4 sqrt(nb) + 32 does the same for the
+exponentials, the row sum and the division, and holds the float32 rounding of either stored
+score. A float32 evaluation of both scorers stays inside the bound, and a 1e-4 relative
+error of the logit scale does not (tests/test_parity_rule.py).
+
+Kept-list rule (top-p lists, per row), with the oracle's selection from its own float32
+scores as the expected list:
+  * bit-exact lists pass ('exact');
+  * the cut may differ only where the oracle's float32 cumulative mass at the cut lies within
+    WINDOW (1e-5) of p ('window');
+  * entries may differ only position by position, and only between two blocks whose oracle
+    scores are closer than the sum of their error bounds: the kernel's arithmetic cannot
+    order them ('tie'; 'window_tie' when the cut moved as well).
+Anything else is a true mismatch; the gate is zero true mismatches, and the tests report and
+bound the exempted rows.
 """
 from __future__ import annotations
+
+import math
 
 import numpy as np
 import torch
@@ -17,11 +48,13 @@ import torch
 from oracle import bsa_oracle as O
 
 WINDOW = 1e-5
-# Relative error bound of a float32 block score: logits |x| <= ~60 carry <= ~1e-5 absolute
-# float32 error after a 128-term dot product, i.e. <= ~2e-5 relative after exp; the bound
-# below keeps a 2.5x margin.
-TIE_REL = 5e-5
-TIE_ABS = 1e-12
+U32 = 2.0 ** -24
+K_DOT = 4.0
+K_POOL = 4.0
+
+
+def k_norm(nb: int) -> float:
+    return 4.0 * math.sqrt(nb) + 32.0
 
 
 def to_dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -36,16 +69,53 @@ def bf16_bits_f64(bits):
     return O.bf16_to_f64(bits)
 
 
+# ------------------------------------------------------------------ score error bound
+
+def score_bound(Qh: np.ndarray, Kh: np.ndarray, layout, mode: str, S: np.ndarray | None = None) -> np.ndarray:
+    """Absolute error bound [nb, nb] of a float32 kernel's block scores for one head
+    (float64 Q, K [N, d] in raster order); S are the exact scores if already computed."""
+    d = Qh.shape[1]
+    s = 1.0 / math.sqrt(d)
+    kbar = O.pool_blocks(Kh, layout)
+    kabs = O.pool_blocks(np.abs(Kh), layout)
+    nb = layout.nb
+    if mode == "meanpool":
+        qbar = O.pool_blocks(Qh, layout)
+        qabs = O.pool_blocks(np.abs(Qh), layout)
+        E = s * (K_DOT * (np.abs(qbar) @ np.abs(kbar).T)
+                 + K_POOL * (qabs @ np.abs(kbar).T + np.abs(qbar) @ kabs.T))
+        if S is None:
+            S = O.score_meanpool(Qh, Kh, layout)
+        return S * U32 * (E + (S * E).sum(axis=1, keepdims=True) + k_norm(nb))
+    if mode == "park":
+        out = np.zeros((nb, nb))
+        ak, akk = np.abs(kbar).T, kabs.T
+        for i in range(nb):
+            q = Qh[layout.rows(i)]
+            x = q @ kbar.T * s
+            p = np.exp(x - x.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            aq = np.abs(q)
+            E = s * (K_DOT * (aq @ ak) + K_POOL * (aq @ akk))
+            out[i] = (p * U32 * (E + (p * E).sum(axis=1, keepdims=True))).mean(axis=0) + p.mean(axis=0) * U32 * k_norm(nb)
+        return out
+    raise ValueError(mode)
+
+
+# ------------------------------------------------------------------ kept-list rule
+
 def _expected(order, m, forced):
     keep = set(order[:m].tolist()) | set(forced)
     return [int(j) for j in order if int(j) in keep]
 
 
-def compare_row(gpu_list, scores_f32, p, forced, text_row):
-    """Classify one row: 'exact', 'window', 'tie' or 'mismatch'."""
+def compare_row(gpu_list, scores_f32, bound, p, forced, text_row):
+    """Classify one row: 'exact', 'window', 'tie', 'window_tie' or 'mismatch'.
+    `bound` holds the score error bound of every block of the row (None: no near-ties)."""
     s = np.asarray(scores_f32, np.float32)
     n = len(s)
-    kept_o, order, cum = O.select_row(s, 1.0 if text_row else p, forced)
+    p_eff = 1.0 if text_row else p
+    kept_o, order, cum = O.select_row(s, p_eff, forced)
     g = [int(x) for x in gpu_list]
     if g == kept_o:
         return "exact"
@@ -53,33 +123,35 @@ def compare_row(gpu_list, scores_f32, p, forced, text_row):
         return "mismatch"
     if text_row or p >= 1.0:
         allowed = [n]
+        m_oracle = n
     else:
         p32 = np.float32(p)
+        hit = np.nonzero(cum >= p32)[0]
+        m_oracle = int(hit[0]) + 1 if len(hit) else n
         allowed = [m for m in range(1, n + 1)
                    if cum[m - 1] >= p32 - WINDOW and (m == 1 or cum[m - 2] < p32 + WINDOW)]
-    for m in allowed:
-        if g == _expected(order, m, forced):
-            return "window"
     s64 = s.astype(np.float64)
-    for m in allowed + [len(g)]:
+    for m in allowed:
         e = _expected(order, m, forced)
         if len(e) != len(g):
             continue
-        ok = True
-        for a, b in zip(g, e):
-            if a != b and abs(s64[a] - s64[b]) > TIE_REL * max(s64[a], s64[b]) + TIE_ABS:
-                ok = False
-                break
-        if ok:
-            return "tie"
+        diffs = [(a, b) for a, b in zip(g, e) if a != b]
+        if diffs and bound is None:
+            continue
+        if all(abs(s64[a] - s64[b]) <= bound[a] + bound[b] for a, b in diffs):
+            moved = m != m_oracle
+            if not diffs:
+                return "window"
+            return "window_tie" if moved else "tie"
     return "mismatch"
 
 
-def compare_masks(gpu_idx, gpu_cnt, scores_f32, p_heads, layout, heads=None):
-    """Compare every row of the GPU kept lists against the oracle's selection from the
-    given float32 scores [heads, nb, nb]. Returns a dict of counts and the first
-    mismatches."""
-    counts = {"exact": 0, "window": 0, "tie": 0, "mismatch": 0}
+def compare_masks(gpu_idx, gpu_cnt, scores_f32, p_heads, layout, heads=None, bounds=None):
+    """Compare every row of the GPU kept lists against the oracle's selection from the given
+    float32 scores [heads, nb, nb]; `bounds` [heads, nb, nb] are the score error bounds (None:
+    identical scores on both sides, no near-tie exemption). Returns a dict of counts and the
+    first mismatches."""
+    counts = {"exact": 0, "window": 0, "tie": 0, "window_tie": 0, "mismatch": 0}
     bad = []
     text = list(range(layout.nb_video, layout.nb))
     for h in (range(scores_f32.shape[0]) if heads is None else heads):
@@ -87,13 +159,23 @@ def compare_masks(gpu_idx, gpu_cnt, scores_f32, p_heads, layout, heads=None):
             c = int(gpu_cnt[h, i])
             row = gpu_idx[h, i, :max(c, 0)]
             text_row = layout.is_text_block(i)
-            kind = compare_row(row, scores_f32[h, i], float(p_heads[h]),
-                               [] if text_row else text, text_row)
+            kind = compare_row(row, scores_f32[h, i], None if bounds is None else bounds[h][i],
+                               float(p_heads[h]), [] if text_row else text, text_row)
             counts[kind] += 1
             if kind == "mismatch" and len(bad) < 5:
                 bad.append((h, i, row.tolist()[:12]))
+    counts["rows"] = sum(counts[k] for k in ("exact", "window", "tie", "window_tie", "mismatch"))
+    counts["exempt"] = counts["window"] + counts["tie"] + counts["window_tie"]
     counts["first_mismatches"] = bad
     return counts
+
+
+def exempt_limit(rows: int) -> int:
+    """Largest number of exempted rows a parity test accepts: near-ties and cuts within 1e-5
+    of p are rare on these inputs (a row needs two scores within ~1e-6 of each other, or a
+    cumulative mass within 1e-5 of p), so more than 0.5% of the rows (at least 2) would say
+    the rule is hiding real differences."""
+    return max(2, rows // 200)
 
 
 def attention_errors(gpu_o, ref_o, rows):

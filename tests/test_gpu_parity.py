@@ -1,10 +1,12 @@
 """CUDA path vs the CPU oracle on the same seeded inputs, call by call, through the C ABI.
 
-Tolerances (stated by the task's parity rule for bf16 inputs with fp32 accumulation):
-attention max-abs <= 3e-2 and relative-L2 <= 1e-2 on the oracle's mask; kept lists
-bit-exact except rows the comparison rule in tests/parity.py exempts; scores within the
-float32 error bound of the scorer."""
+Tolerances: attention max-abs <= 3e-2 and relative-L2 <= 1e-2 on the oracle's mask (bf16
+inputs, float32 accumulation); scores within the float32 error bound of tests/parity.py
+(score_bound), element by element; kept lists bit-exact except the rows the comparison rule
+of tests/parity.py exempts (a cut within 1e-5 of p, or two blocks closer than their score
+bounds), whose number every mask test prints and bounds."""
 import math
+import os
 
 import numpy as np
 import pytest
@@ -18,8 +20,6 @@ pytestmark = pytest.mark.gpu
 
 ATT_MAX_ABS = 3e-2
 ATT_REL_L2 = 1e-2
-SCORE_RTOL = 5e-5      # float32 scorer vs float64 oracle, relative (see parity.TIE_REL)
-SCORE_ATOL = 1e-7
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -41,7 +41,9 @@ class Case:
     def __init__(self, heads, d, T, H, W, text, B, p, mode="meanpool", seed=0, tile=(0, 0, 0)):
         bsa = _bsa()
         self.heads, self.d, self.B = heads, d, B
-        self.Qb, self.Kb, self.Vb = inputs.generate_qkv(heads, d, T, H, W, text, seed)
+        big = heads * (T * H * W + text) > 4_000_000
+        self.Qb, self.Kb, self.Vb = inputs.generate_qkv(heads, d, T, H, W, text, seed,
+                                                        workers=min(os.cpu_count() or 1, 16) if big else 1)
         self.N = self.Qb.shape[1]
         self.p = np.array([p] * heads if np.isscalar(p) else p, dtype=np.float64)
         self.mode = mode
@@ -80,6 +82,26 @@ class Case:
     def oracle_scores(self, h):
         return O.score_head(O.bf16_to_f64(self.Qb[h]), O.bf16_to_f64(self.Kb[h]), self.layout, self.mode)
 
+    def oracle_scores_and_bound(self, h):
+        """Exact scores (float64) of head h and the float32 kernel's error bound on them."""
+        Qh, Kh = O.bf16_to_f64(self.Qb[h]), O.bf16_to_f64(self.Kb[h])
+        S = O.score_head(Qh, Kh, self.layout, self.mode)
+        return S, PT.score_bound(Qh, Kh, self.layout, self.mode, S if self.mode == "meanpool" else None)
+
+
+def _check_scores(S_gpu_h, S, bnd, where):
+    err = np.abs(S_gpu_h.astype(np.float64) - S)
+    worst = float((err / bnd).max())
+    print(f"\n[score bound] {where}: worst |error| / bound = {worst:.3f}")
+    assert worst <= 1.0, (where, worst, float(err.max()))
+    assert np.allclose(S_gpu_h.sum(axis=1), 1.0, atol=1e-5)
+    return worst
+
+
+def _report(tag, res):
+    print(f"\n[mask parity] {tag}: rows={res['rows']} exact={res['exact']} window={res['window']} "
+          f"tie={res['tie']} window_tie={res['window_tie']} mismatch={res['mismatch']}")
+
 
 def _status_ok():
     assert _bsa().bsa_device_status() == 0
@@ -93,6 +115,8 @@ SMALL = {
     "text_d64_b128": dict(heads=3, d=64, T=5, H=11, W=13, text=200, B=128, p=0.9),
     # d=128, B=128 with text, several tiles and a partial last video block
     "text_d128_b128": dict(heads=2, d=128, T=6, H=20, W=24, text=256, B=128, p=0.95),
+    # a grid smaller than one block: nb = 1, one partial block (63 real tokens)
+    "single_block": dict(heads=2, d=64, T=1, H=7, W=9, text=0, B=64, p=0.9),
 }
 
 
@@ -104,10 +128,8 @@ def test_scores_match_oracle(name, mode):
     torch.cuda.synchronize()
     _status_ok()
     for h in range(c.heads):
-        ref = c.oracle_scores(h)
-        err = np.abs(S[h] - ref)
-        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * ref), (h, float(err.max()))
-        assert np.allclose(S[h].sum(axis=1), 1.0, atol=1e-5)
+        ref, bnd = c.oracle_scores_and_bound(h)
+        _check_scores(S[h], ref, bnd, (name, mode, h))
 
 
 # Enough 128-row items (heads x query tiles >= SM count) that the mean-pooled scores take the
@@ -125,10 +147,8 @@ def test_scores_tensor_core_path_match_oracle(name):
     torch.cuda.synchronize()
     _status_ok()
     for h in range(0, c.heads, 7):
-        ref = c.oracle_scores(h)
-        err = np.abs(S[h] - ref)
-        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * ref), (h, float(err.max()))
-        assert np.allclose(S[h].sum(axis=1), 1.0, atol=1e-5)
+        ref, bnd = c.oracle_scores_and_bound(h)
+        _check_scores(S[h], ref, bnd, (name, h))
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -139,8 +159,9 @@ def test_select_on_oracle_scores_is_exact(name):
     idx, cnt = c.gpu_select(torch.from_numpy(S).cuda())
     _status_ok()
     res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, c.p, c.layout)
-    assert res["mismatch"] == 0 and res["tie"] == 0, res
-    assert res["exact"] >= (c.heads * c.nb) - 2, res
+    _report(f"select on oracle scores, {name}", res)
+    assert res["mismatch"] == 0 and res["tie"] == 0 and res["window_tie"] == 0, res
+    assert res["window"] <= PT.exempt_limit(res["rows"]), res
 
 
 @pytest.mark.parametrize("p", [1.0, 1e-6, 0.5])
@@ -154,7 +175,8 @@ def test_select_edge_p(p):
     if p == 1e-6:
         assert (cnt[:, :c.layout.nb_video] == 1 + c.layout.nb_text).all()
     res = PT.compare_masks(idx.cpu().numpy(), cnt, S, c.p, c.layout)
-    assert res["mismatch"] == 0 and res["tie"] == 0, res
+    assert res["mismatch"] == 0 and res["tie"] == 0 and res["window_tie"] == 0, res
+    assert res["window"] <= PT.exempt_limit(res["rows"]), res
 
 
 def test_select_hand_rows():
@@ -188,9 +210,13 @@ def test_masks_end_to_end(name, mode):
     c = Case(**SMALL[name], mode=mode)
     idx, cnt = c.gpu_select(c.gpu_scores())
     _status_ok()
-    S = np.stack([c.oracle_scores(h).astype(np.float32) for h in range(c.heads)])
-    res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, c.p, c.layout)
+    sb = [c.oracle_scores_and_bound(h) for h in range(c.heads)]
+    S = np.stack([x[0].astype(np.float32) for x in sb])
+    res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, c.p, c.layout,
+                           bounds=[x[1] for x in sb])
+    _report(f"end to end, {name}, {mode}", res)
     assert res["mismatch"] == 0, res
+    assert res["exempt"] <= PT.exempt_limit(res["rows"]), res
 
 
 def _oracle_mask(c):
@@ -336,7 +362,7 @@ def _full_case(name, mode="meanpool"):
 @pytest.mark.slow
 @pytest.mark.parametrize("name,mode", [("wan13b_480p", "meanpool"), ("wan13b_480p", "park"),
                                        ("wan14b_720p", "meanpool"), ("wan14b_720p", "park"),
-                                       ("hunyuan_720p", "meanpool")])
+                                       ("hunyuan_720p", "meanpool"), ("hunyuan_720p", "park")])
 def test_full_size_masks_and_sampled_attention(name, mode):
     c = _full_case(name, mode)
     S_gpu = c.gpu_scores()
@@ -347,12 +373,15 @@ def test_full_size_masks_and_sampled_attention(name, mode):
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
     rng = np.random.default_rng(0)
     S_or = np.zeros_like(S_gpu)
+    bounds = {}
     for h in heads:
-        S_or[h] = c.oracle_scores(h).astype(np.float32)
-        err = np.abs(S_gpu[h] - S_or[h])
-        assert np.all(err <= SCORE_ATOL + SCORE_RTOL * S_or[h]), (h, float(err.max()))
-    res = PT.compare_masks(idx_h, cnt_h, S_or, c.p, c.layout, heads=heads)
+        ref, bounds[h] = c.oracle_scores_and_bound(h)
+        S_or[h] = ref.astype(np.float32)
+        _check_scores(S_gpu[h], ref, bounds[h], (name, mode, h))
+    res = PT.compare_masks(idx_h, cnt_h, S_or, c.p, c.layout, heads=heads, bounds=bounds)
+    _report(f"full size, {name}, {mode}, heads {heads}", res)
     assert res["mismatch"] == 0, res
+    assert res["exempt"] <= PT.exempt_limit(res["rows"]), res
     # attention on the oracle's mask for sampled query blocks (text rows included)
     oi = {h: O.select_topp(S_or[h], c.p[h], c.layout) for h in heads}
     idx_o = idx.clone()
@@ -393,6 +422,7 @@ def test_select_flat_and_peaked_rows(conc, p):
     bsa.bsa_select_topp(prob, torch.from_numpy(S).cuda(), pd, None, idx, cnt)
     _status_ok()
     res = PT.compare_masks(idx.cpu().numpy(), cnt.cpu().numpy(), S, np.full(heads, p), L)
-    assert res["mismatch"] == 0 and res["tie"] == 0, res
+    assert res["mismatch"] == 0 and res["tie"] == 0 and res["window_tie"] == 0, res
+    assert res["window"] <= PT.exempt_limit(res["rows"]), res
     if conc >= 5.0:
         assert cnt.cpu().numpy().mean() > 64       # the fallback path was exercised

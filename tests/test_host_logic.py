@@ -1,7 +1,8 @@
 """Host-side logic with no GPU: workspace sizes cover every buffer the kernels address, and
-bench.py's roofline traffic is taken from the committed ncu summary only while the kernel
-sources it was measured on are unchanged."""
+bench.py's roofline traffic is taken from the committed ncu figures (profiles/*.json) only
+while the kernel sources they were measured on are unchanged."""
 import importlib.util
+import json
 import os
 import shutil
 
@@ -48,19 +49,23 @@ def _load_bench(root):
 
 def test_profiled_traffic_only_for_matching_sources(tmp_path):
     bench = _load_bench(ROOT)
-    t = bench._profiled_traffic("sparse_attention", "wan13b_480p")
-    assert t is None or (isinstance(t, int) and t > 0)
     assert bench._profiled_traffic("sparse_attention", "no_such_workload") is None
-    assert bench._profiled_traffic("drift_check", "wan13b_480p") is None
-    # a copy of the tree whose kernel source differs by one byte gets no traffic figure
+    assert bench._profiled_traffic("drift_check", "hunyuan_720p") is None
+    # a copy of the tree with a profile written for its current kernel sources
     csrc = os.path.join("block_sparse_attention_query_b200", "csrc")
     os.makedirs(tmp_path / csrc)
+    os.makedirs(tmp_path / "profiles")
     shutil.copy(os.path.join(ROOT, "bench.py"), tmp_path / "bench.py")
-    shutil.copytree(os.path.join(ROOT, "profiles"), tmp_path / "profiles")
     for f in ("attention.cuh", "bsa_common.cuh"):
         shutil.copy(os.path.join(ROOT, csrc, f), tmp_path / csrc / f)
     copy = _load_bench(str(tmp_path))
-    assert copy._profiled_traffic("sparse_attention", "wan13b_480p") == t
+    rec = {"workload": "hunyuan_720p", "traffic_bytes_per_launch": 123456789,
+           "sources_sha256_16": copy._sources_hash(str(tmp_path))}
+    with open(tmp_path / "profiles" / "sparse_attention_hunyuan_720p.json", "w") as f:
+        json.dump(rec, f)
+    assert copy._profiled_traffic("sparse_attention", "hunyuan_720p") == 123456789
+    assert copy._profiled_traffic("sparse_attention", "wan13b_480p") is None
+    # one byte more in a kernel source: the figure is stale and is not used
     with open(tmp_path / csrc / "attention.cuh", "a") as f:
         f.write("\n")
-    assert copy._profiled_traffic("sparse_attention", "wan13b_480p") is None
+    assert copy._profiled_traffic("sparse_attention", "hunyuan_720p") is None

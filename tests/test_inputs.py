@@ -40,3 +40,13 @@ def test_workloads():
     assert w.heads == 40 and len(w.p) == 40 and set(w.p) <= set(inputs.TOP_P_CHOICES)
     assert inputs.workload("hunyuan_720p").tokens == 119056
     assert inputs.workload("wan13b_480p").tokens == 32760
+
+
+def test_head_ranges_draw_the_same_heads():
+    # one GPU's share of the heads (or heads drawn in parallel) equals that slice of the layer
+    full = inputs.generate_qkv(5, 16, 2, 3, 4, 5, seed=3)
+    part = inputs.generate_qkv(5, 16, 2, 3, 4, 5, seed=3, head_range=(2, 4))
+    par = inputs.generate_qkv(5, 16, 2, 3, 4, 5, seed=3, workers=3)
+    for x, y, z in zip(full, part, par):
+        assert np.array_equal(x[2:4], y)
+        assert np.array_equal(x, z)
