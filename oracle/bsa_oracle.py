@@ -16,6 +16,8 @@ the slow, obvious way, in the order the pages describe the method:
 5. ``drift``           — per-head relative Q/K change since the cached reference
 6. ``sparse_attention``— exact softmax attention restricted to the kept key blocks
 7. ``reuse_run``       — the drift-gated mask-reuse loop across denoising steps
+8. ``captured_mass``   — retrieval accuracy: the share of each query's exact (dense)
+   attention mass that falls on its kept key blocks
 
 Sources (page title, then the part of the page):
 * PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers —
@@ -31,6 +33,9 @@ Sources (page title, then the part of the page):
 * RAPID: Reusing Attention Sparsity with Inter-step Adaptation for Efficient Video
   Diffusion — English abstract: 3D attention, block importance estimated and the sparse
   mask cached for reuse across steps.
+* PARK — Abstract: inaccurate block retrieval either degrades quality or wastes computation;
+  PARK is judged by its block retrieval accuracy (``captured_mass`` measures it without a
+  model: how much of the exact attention the retrieved blocks hold).
 
 Where the pages are silent the plainest reading is taken; each one is named at the point
 of use (block shape/order, logit scale, top-p boundary, tie order, text blocks, drift
@@ -338,4 +343,34 @@ def reuse_run(steps_qk, V, layout, p, tau, mode="meanpool", attend=True):
         if attend:
             out["O"].append(np.stack(Os))
     out["masks"] = masks
+    return out
+
+
+# ------------------------------------------------------------------ 8. retrieval accuracy
+
+def captured_mass(Qh, Kh, idx, cnt, layout: Layout, qblocks=None) -> np.ndarray:
+    """Share of the exact attention mass that each query block's kept key blocks capture.
+
+    For a real query t of block i, its exact attention is softmax over ALL real keys u of
+    Q_t . K_u / sqrt(d); the captured mass is the sum of that distribution over the real keys
+    of the kept blocks idx[i, :cnt[i]] (PARK abstract: accurate block retrieval, where an
+    inaccurate retrieval loses attention mass or spends computation on blocks that hold
+    little). Returned per query block, as the mean over its real queries: float64 [nb]
+    (NaN for blocks not in `qblocks`). Reading: the plain average over queries, every query
+    weighted alike.
+    """
+    d = Qh.shape[1]
+    scale = 1.0 / math.sqrt(d)
+    real = np.concatenate([layout.rows(j) for j in range(layout.nb)])
+    out = np.full(layout.nb, np.nan)
+    for i in (range(layout.nb) if qblocks is None else qblocks):
+        rows = layout.rows(i)
+        L = (Qh[rows] @ Kh[real].T) * scale
+        m = L.max(axis=1, keepdims=True)
+        e = np.exp(L - m)
+        p = e / e.sum(axis=1, keepdims=True)
+        kept = np.zeros(Qh.shape[0], dtype=bool)
+        for j in idx[i, :cnt[i]]:
+            kept[layout.rows(int(j))] = True
+        out[i] = p[:, kept[real]].sum(axis=1).mean()
     return out

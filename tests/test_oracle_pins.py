@@ -308,3 +308,67 @@ def test_reuse_run_refreshes_when_drift_exceeds_tau():
     out = O.reuse_run([(q0, k0), (q0, k0), (q2, k0), (q2, k0)], V, L, [0.9], 0.05)
     assert [r[0] for r in out["refresh"]] == [True, False, True, False]
     assert out["drift"][2][0] == pytest.approx(1.0, abs=1e-15)
+
+
+# --------------------------------------------------------------------- retrieval accuracy
+
+def _mass_case(T=2, H=8, W=12, text=20, B=16, tile=(1, 4, 4), d=8, seed=11):
+    rng = np.random.default_rng(seed)
+    L = O.block_layout(T, H, W, text, B, tile)
+    N = T * H * W + text
+    Q = _bf16_round_f64(rng.standard_normal((N, d)) * 1.5)
+    K = _bf16_round_f64(rng.standard_normal((N, d)) * 1.5)
+    return L, Q, K
+
+
+def test_captured_mass_all_blocks_is_one():
+    L, Q, K = _mass_case()
+    idx = np.tile(np.arange(L.nb, dtype=np.int32), (L.nb, 1))
+    cnt = np.full(L.nb, L.nb, np.int32)
+    assert np.allclose(O.captured_mass(Q, K, idx, cnt, L), 1.0, atol=1e-12)
+
+
+def test_captured_mass_equals_brute_force_softmax():
+    # torch's softmax over the full logits, summed over the kept keys' columns
+    L, Q, K = _mass_case()
+    rng = np.random.default_rng(2)
+    idx = np.full((L.nb, L.nb), -1, np.int32)
+    cnt = rng.integers(1, L.nb + 1, L.nb).astype(np.int32)
+    for i in range(L.nb):
+        idx[i, :cnt[i]] = rng.permutation(L.nb)[:cnt[i]]
+    got = O.captured_mass(Q, K, idx, cnt, L)
+    P = torch.softmax(torch.from_numpy(Q @ K.T / math.sqrt(Q.shape[1])), dim=1).numpy()
+    for i in range(L.nb):
+        rows = L.rows(i)
+        cols = np.concatenate([L.rows(int(j)) for j in idx[i, :cnt[i]]])
+        assert got[i] == pytest.approx(P[np.ix_(rows, cols)].sum(axis=1).mean(), abs=1e-12)
+
+
+def test_captured_mass_with_constant_keys_is_sum_of_park_scores():
+    # keys constant within every block: PARK's score of block j is the exact mass of j, so the
+    # captured mass is the sum of the kept blocks' PARK scores (and is additive over blocks)
+    L, Q, K = _mass_case(text=0, B=16)
+    rng = np.random.default_rng(4)
+    for j in range(L.nb):
+        K[L.rows(j)] = _bf16_round_f64(rng.standard_normal(K.shape[1]))
+    P = O.score_park(Q, K, L)
+    idx = np.full((L.nb, L.nb), -1, np.int32)
+    cnt = np.zeros(L.nb, np.int32)
+    for i in range(L.nb):
+        keep = rng.permutation(L.nb)[:3]
+        idx[i, :3] = keep
+        cnt[i] = 3
+    got = O.captured_mass(Q, K, idx, cnt, L)
+    for i in range(L.nb):
+        assert got[i] == pytest.approx(P[i, idx[i, :3]].sum(), abs=1e-12)
+
+
+def test_captured_mass_grows_with_the_kept_set():
+    L, Q, K = _mass_case()
+    S = O.score_park(Q, K, L).astype(np.float32)
+    prev = np.zeros(L.nb)
+    for p in (0.3, 0.6, 0.9, 1.0):
+        idx, cnt = O.select_topp(S, p, L)
+        m = O.captured_mass(Q, K, idx, cnt, L)
+        assert np.all(m >= prev - 1e-12) and np.all(m <= 1 + 1e-12)
+        prev = m
