@@ -18,6 +18,8 @@ the slow, obvious way, in the order the pages describe the method:
 7. ``reuse_run``       — the drift-gated mask-reuse loop across denoising steps
 8. ``captured_mass``   — retrieval accuracy: the share of each query's exact (dense)
    attention mass that falls on its kept key blocks
+9. ``rapid_run``       — one-shot block-importance estimate early in the run, cached scores
+   and mask reused for the later steps, optional staged re-selection (Turbo)
 
 Sources (page title, then the part of the page):
 * PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers —
@@ -373,4 +375,64 @@ def captured_mass(Qh, Kh, idx, cnt, layout: Layout, qblocks=None) -> np.ndarray:
         for j in idx[i, :cnt[i]]:
             kept[layout.rows(int(j))] = True
         out[i] = p[:, kept[real]].sum(axis=1).mean()
+    return out
+
+
+# ---------------------------------------------------------------- 9. one-shot schedule
+
+def rapid_run(steps_qk, V, layout, p0, estimate_step=0, stages=(), mode="meanpool", attend=True):
+    """One-shot block-importance estimate with cached reuse, and Turbo staged pruning.
+
+    RAPID English abstract: block importance is estimated once, early in the generation; the
+    scores and the sparse mask are cached and reused by the later steps (no recalculation);
+    the cached scores also allow an optional multi-stage adaptive pruning (Turbo mode), since
+    the attention density the steps need decays as the generation proceeds. Readings (the
+    abstract gives no schedule): steps before `estimate_step` attend densely (every key
+    block); at `estimate_step` every head is scored and its kept lists are selected with p0
+    (per head); `stages` is a sequence of (step, p) with increasing steps: from each such step
+    on, the kept lists are selected anew from the CACHED scores with that p (no re-scoring).
+
+    `steps_qk` yields (Q, K) bf16 bits [heads, N, d] per step; V is fixed. Returns a dict
+    with per-step kept-block counts (None for dense steps), the selection each step used
+    ('dense', 'estimate', 'reuse' or 'stage'), the final masks and scores and (if
+    `attend`) the per-step outputs.
+    """
+    heads = V.shape[0]
+    Vf = [bf16_to_f64(V[h]) for h in range(heads)]
+    stage_p = {int(s): p for s, p in stages}
+    scores = [None] * heads
+    masks = [None] * heads
+    out = {"kind": [], "cnt": [], "O": []}
+    for s, (Q, K) in enumerate(steps_qk):
+        if s < estimate_step:
+            kind = "dense"
+        elif s == estimate_step:
+            kind = "estimate"
+        elif s in stage_p:
+            kind = "stage"
+        else:
+            kind = "reuse"
+        Os, cnts = [], []
+        for h in range(heads):
+            Qh, Kh = bf16_to_f64(Q[h]), bf16_to_f64(K[h])
+            if kind == "estimate":
+                scores[h] = score_head(Qh, Kh, layout, mode).astype(np.float32)
+                masks[h] = select_topp(scores[h], p0[h], layout)
+            elif kind == "stage":
+                masks[h] = select_topp(scores[h], stage_p[s], layout)
+            if kind == "dense":
+                idx = np.tile(np.arange(layout.nb, dtype=np.int32), (layout.nb, 1))
+                cnt = np.full(layout.nb, layout.nb, dtype=np.int32)
+                cnts.append(None)
+            else:
+                idx, cnt = masks[h]
+                cnts.append(cnt.copy())
+            if attend:
+                Os.append(sparse_attention_head(Qh, Kh, Vf[h], idx, cnt, layout))
+        out["kind"].append(kind)
+        out["cnt"].append(cnts)
+        if attend:
+            out["O"].append(np.stack(Os))
+    out["masks"] = masks
+    out["scores"] = scores
     return out

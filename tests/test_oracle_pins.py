@@ -372,3 +372,50 @@ def test_captured_mass_grows_with_the_kept_set():
         m = O.captured_mass(Q, K, idx, cnt, L)
         assert np.all(m >= prev - 1e-12) and np.all(m <= 1 + 1e-12)
         prev = m
+
+
+# --------------------------------------------------------------------- one-shot schedule
+
+def _walk_steps(n, shape=(2, 16, 2, 8, 16, 0, 32), tile=(1, 4, 8)):
+    heads, d, T, H, W, text, B = shape
+    walk = inputs.RandomWalk(heads, d, T, H, W, text, seed=5)
+    steps = []
+    for _ in range(n):
+        q, k, v = walk.current()
+        steps.append((q, k))
+        walk.advance()
+    return steps, v, O.block_layout(T, H, W, text, B, tile)
+
+
+def test_rapid_dense_before_estimate_and_reuse_after():
+    steps, V, L = _walk_steps(5)
+    r = O.rapid_run(steps, V, L, [0.9, 0.8], estimate_step=2)
+    assert r["kind"] == ["dense", "dense", "estimate", "reuse", "reuse"]
+    # dense steps equal dense softmax attention (torch SDPA)
+    for s in (0, 1):
+        for h in range(V.shape[0]):
+            q, k, v = (torch.from_numpy(O.bf16_to_f64(x[h])) for x in (steps[s][0], steps[s][1], V))
+            ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0].numpy()
+            assert np.allclose(r["O"][s][h], ref, atol=1e-10)
+    # the estimate uses the scores of step 2's Q, K; later steps reuse that mask unchanged
+    for h in range(V.shape[0]):
+        S = O.score_meanpool(O.bf16_to_f64(steps[2][0][h]), O.bf16_to_f64(steps[2][1][h]), L).astype(np.float32)
+        idx, cnt = O.select_topp(S, [0.9, 0.8][h], L)
+        assert np.array_equal(r["cnt"][2][h], cnt) and np.array_equal(r["cnt"][4][h], cnt)
+        assert np.array_equal(r["masks"][h][0], idx)
+
+
+def test_rapid_turbo_stages_prune_the_cached_ranking():
+    steps, V, L = _walk_steps(7)
+    r = O.rapid_run(steps, V, L, [0.95, 0.95], estimate_step=0, stages=[(3, 0.8), (5, 0.6)], attend=False)
+    assert r["kind"] == ["estimate", "reuse", "reuse", "stage", "reuse", "stage", "reuse"]
+    for h in range(V.shape[0]):
+        S = r["scores"][h]
+        # each stage keeps a prefix of the same cached ranking, so kept sets only shrink
+        for a, b in ((0, 3), (3, 5)):
+            assert np.all(r["cnt"][b][h] <= r["cnt"][a][h])
+        idx, cnt = O.select_topp(S, 0.6, L)
+        assert np.array_equal(r["cnt"][6][h], cnt)
+        for i in range(L.nb):
+            order = O.sort_row(S[i])
+            assert list(r["masks"][h][0][i, :cnt[i]]) == [int(j) for j in order[:cnt[i]]]
