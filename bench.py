@@ -332,6 +332,8 @@ def run_ours(args, ws, rank, local):
         e2e = {"value": round(e2e_ms, 4), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * H * N * d * elem), "d2h_bytes_per_step": int(H * N * d * elem)}
 
+    retrieval = None if args.no_retrieval else retrieval_accuracy(w, h0, h1, sets[0], dev, ws)
+
     line = {
         "metric": METRIC, "value": round(ms_step, 5), "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -351,11 +353,52 @@ def run_ours(args, ws, rank, local):
         "kept_density": round(kept_pairs / (H * plan.nb * plan.nb), 5),
         "tflops_actual_call": round(att_flops / (ms_step * 1e-3) / 1e12, 2),
         "tflops_dense_equiv_call": round(dense_flops / (ms_step * 1e-3) / 1e12, 2),
-        "stages": stages, "roofline": roof, "e2e": e2e,
+        "stages": stages, "roofline": roof, "e2e": e2e, "retrieval": retrieval,
         "gpu_launches": launches, "gpu_launches_per_step": round(launches / args.steps / ws, 2),
         "clocks": clocks,
     }
     return line, (w, host_sets[0] if (rank == 0 and ws == 1) else None)
+
+
+def retrieval_accuracy(w, h0, h1, qkv, dev, ws):
+    """Retrieval accuracy of both scorers on this rank's heads (outside the timed region): the
+    captured mass of their top-p masks (the share of each query's exact attention that the
+    kept blocks hold), averaged over all query blocks of all heads, and their kept density."""
+    import torch
+
+    from block_sparse_attention_query_b200 import bsa
+    Q, K, _ = qkv
+    Hl = h1 - h0
+    p = torch.tensor(list(w.p[h0:h1]), dtype=torch.float32, device=dev)
+    out = {}
+    for name, mode in (("meanpool", bsa.BSA_SCORE_MEANPOOL), ("park", bsa.BSA_SCORE_PARK)):
+        prob = bsa.problem(Hl, w.d, w.T, w.H, w.W, w.text_tokens, w.block, score_mode=mode)
+        plan = bsa.bsa_plan(prob)
+        nb = plan.nb
+        S = torch.empty(Hl, nb, nb, dtype=torch.float32, device=dev)
+        idx = torch.empty(Hl, nb, nb, dtype=torch.int32, device=dev)
+        cnt = torch.empty(Hl, nb, dtype=torch.int32, device=dev)
+        mass = torch.empty(Hl, nb, dtype=torch.float32, device=dev)
+        bsa.bsa_score_blocks(prob, Q, K, None, S, torch.empty(plan.score_workspace_bytes, dtype=torch.uint8, device=dev))
+        bsa.bsa_select_topp(prob, S, p, None, idx, cnt)
+        wsm = torch.empty(plan.mass_workspace_bytes, dtype=torch.uint8, device=dev)
+        bsa.bsa_captured_mass(prob, Q, K, idx, cnt, mass, wsm)
+        del wsm
+        torch.cuda.synchronize()
+        st = bsa.bsa_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} in the retrieval measurement")
+        vid = mass[:, :plan.nb_video].double()
+        tot = sum_over_ranks(float(vid.sum()), ws, dev)
+        n = sum_over_ranks(float(vid.numel()), ws, dev)
+        kept = sum_over_ranks(float(cnt[:, :plan.nb_video].double().sum()), ws, dev)
+        mn = float(vid.min()) if ws == 1 else None
+        out[name] = {"captured_mass_mean": round(tot / n, 5), "kept_blocks_per_video_row": round(kept / n, 3)}
+        if mn is not None:
+            out[name]["captured_mass_min_block"] = round(mn, 5)
+    out["definition"] = ("mean over video query blocks of the share of each query's exact softmax mass held by "
+                         "its top-p kept blocks (bsa_captured_mass)")
+    return out
 
 
 # ------------------------------------------------------------------------- oracle
@@ -433,15 +476,27 @@ def run_reference(args):
     }
 
 
+def turbo_stages(n_steps, p_base):
+    """Default Turbo stages of the one-shot schedule (the page gives none): re-select from the
+    cached scores at 40% and 70% of the run with p lowered by 0.05 and 0.10."""
+    return [(max(1, round(0.4 * n_steps)), round(p_base - 0.05, 4)),
+            (max(2, round(0.7 * n_steps)), round(p_base - 0.10, 4))]
+
+
 def run_reuse(args):
-    """The 50-step reuse run: Q/K random-walk across denoising steps, each head's mask
-    recomputed only when its drift since the last refresh exceeds TAU. Reports amortised ms per
-    step (CUDA events around all steps; all steps' inputs resident before timing) and the
-    refresh count."""
+    """A multi-step run on a Q/K random walk (x_{s+1} = x_s + 0.02 N(0,1), V fixed) under one
+    of the mask schedules:
+      tmr      drift-gated reuse: a head's mask is recomputed only when its drift since the
+               last refresh exceeds TAU (HEART abstract, Temporal Mask Reuse);
+      oneshot  one estimate at --estimate-step (dense attention before it), the cached mask
+               reused by every later step (RAPID English abstract);
+      turbo    oneshot plus staged re-selection from the cached scores with smaller p.
+    Reports amortised ms per step (CUDA events around all steps; all steps' inputs resident
+    before timing) and what the steps did."""
     import torch
 
     from block_sparse_attention_query_b200 import inputs
-    from block_sparse_attention_query_b200.layer import SparseAttentionLayer
+    from block_sparse_attention_query_b200.layer import OneShotLayer, SparseAttentionLayer
 
     w = inputs.workload(args.workload)
     walk = inputs.RandomWalk(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, seed=0)
@@ -456,18 +511,34 @@ def run_reuse(args):
     V = to_dev(v)
     O = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device=dev)
     flags = torch.zeros(args.reuse, w.heads, dtype=torch.int32, device=dev)
+    kept = torch.zeros(args.reuse, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
+    stages = turbo_stages(args.reuse, float(np.mean(w.p))) if args.schedule == "turbo" else []
+    kinds = []
+
+    def make_layer():
+        if args.schedule == "tmr":
+            return SparseAttentionLayer(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, p=list(w.p),
+                                        tau=TAU, device=dev)
+        return OneShotLayer(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, p=list(w.p),
+                            estimate_step=args.estimate_step, stages=stages, device=dev)
 
     def run(timed):
-        layer = SparseAttentionLayer(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block, p=list(w.p),
-                                     tau=TAU, device=dev)
+        layer = make_layer()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         a.record(stream)
         for s in range(args.reuse):
             layer.step(qs[s], ks[s], V, O)
             if timed:
-                flags[s].copy_(layer.refresh)
+                if args.schedule == "tmr":
+                    flags[s].copy_(layer.refresh)
+                    kept[s] = layer.cnt.sum()
+                else:
+                    if len(kinds) < args.reuse:
+                        kinds.append(layer.kind)
+                    if layer.kind != "dense":
+                        kept[s] = layer.cnt.sum()
         b.record(stream)
         torch.cuda.synchronize()
         return a.elapsed_time(b)
@@ -476,17 +547,26 @@ def run_reuse(args):
         run(False)
     ms = [run(True) for _ in range(args.steps)]
     per_step = float(np.median(ms)) / args.reuse
-    refreshes = int(flags.sum().item())
-    return {
-        "metric": "amortised ms per denoising step (50-step reuse run)", "value": round(per_step, 5), "unit": UNIT,
+    from block_sparse_attention_query_b200 import bsa
+    nb = bsa.bsa_plan(bsa.problem(w.heads, w.d, w.T, w.H, w.W, w.text_tokens, w.block)).nb
+    line = {
+        "metric": f"amortised ms per denoising step ({args.reuse}-step {args.schedule} run)",
+        "value": round(per_step, 5), "unit": UNIT,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step, 5),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic random walk x_{s+1} = x_s + 0.02 N(0,1) on Q, K (V fixed)",
-        "config": {"workload": f"{w.name} reuse run", "denoising_steps": args.reuse, "tau": TAU,
-                   "timed_runs": args.steps, "statistic": "median over timed runs"},
-        "refreshes": refreshes, "head_steps": args.reuse * w.heads,
-        "refreshed_per_step": [int(x) for x in flags.sum(dim=1).cpu().tolist()],
+        "config": {"workload": f"{w.name} {args.schedule} run", "denoising_steps": args.reuse,
+                   "schedule": args.schedule, "timed_runs": args.steps, "statistic": "median over timed runs"},
+        "kept_blocks_per_row_per_step": [round(float(x) / (w.heads * nb), 3) for x in kept.cpu().tolist()],
     }
+    if args.schedule == "tmr":
+        line["config"]["tau"] = TAU
+        line.update({"refreshes": int(flags.sum().item()), "head_steps": args.reuse * w.heads,
+                     "refreshed_per_step": [int(x) for x in flags.sum(dim=1).cpu().tolist()]})
+    else:
+        line["config"].update({"estimate_step": args.estimate_step, "stages": stages})
+        line["step_kinds"] = kinds
+    return line
 
 
 def main():
@@ -500,12 +580,16 @@ def main():
     ap.add_argument("--gather", action="store_true", help="all-gather O over the ranks every step (N > 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-retrieval", action="store_true", help="skip the retrieval-accuracy measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU seconds the oracle sample runs for (whole heads, at least one)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (None if stale)")
     ap.add_argument("--reuse", type=int, default=0,
-                    help="run the N-step drift-gated reuse run instead (amortised ms per step)")
+                    help="run an N-step random-walk run under --schedule instead (amortised ms per step)")
+    ap.add_argument("--schedule", default="tmr", choices=["tmr", "oneshot", "turbo"],
+                    help="mask schedule of the --reuse run: drift-gated reuse, one-shot estimate, one-shot + Turbo")
+    ap.add_argument("--estimate-step", type=int, default=0, help="step of the one-shot estimate (oneshot/turbo)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank, local = _dist()

@@ -46,6 +46,7 @@ class PlanInfo(ctypes.Structure):
         ("score_workspace_bytes", ctypes.c_size_t),
         ("drift_workspace_bytes", ctypes.c_size_t),
         ("attention_workspace_bytes", ctypes.c_size_t),
+        ("mass_workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -70,6 +71,12 @@ EXPORTS = {
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                             ctypes.c_void_p]),
+    "bsa_dense_correction": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "bsa_captured_mass": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.c_void_p]),
     "bsa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bsa_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_version": (ctypes.c_char_p, []),
@@ -166,6 +173,18 @@ def bsa_sparse_attention(prob, Q, K, V, idx, cnt, O, ws, stream=None):
                                    _ptr(O), _ptr(ws),
                                    ws.numel() * ws.element_size() if ws is not None else 0,
                                    _stream(stream)), "bsa_sparse_attention")
+
+
+def bsa_dense_correction(prob, Q, K, V, refresh, O, R, ws, stream=None):
+    check(lib.bsa_dense_correction(ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(V), _ptr(refresh), _ptr(O), _ptr(R),
+                                   _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
+                                   _stream(stream)), "bsa_dense_correction")
+
+
+def bsa_captured_mass(prob, Q, K, idx, cnt, mass, ws, stream=None):
+    check(lib.bsa_captured_mass(ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(idx), _ptr(cnt), _ptr(mass), _ptr(ws),
+                                ws.numel() * ws.element_size() if ws is not None else 0,
+                                _stream(stream)), "bsa_captured_mass")
 
 
 def bsa_device_status(stream=None) -> int:

@@ -90,10 +90,13 @@ struct Params {
     const bsa_bf16* Q;
     const bsa_bf16* K;
     const bsa_bf16* V;
-    const int* idx;
+    const int* idx;     // kept lists; idx == cnt == nullptr: every block, in index order
     const int* cnt;
+    const int* head_mask;   // nullable: heads with head_mask[h] == 0 are skipped, nothing written
     const int* perm;    // [nb*B] raster token of every block slot, -1 = padding
     bsa_bf16* O;
+    float* lse;         // nullable, [heads][N]: log2 of the row's softmax denominator in log2
+                        // units of the scaled logits (-inf when nothing is kept)
     float* part_o;      // [n_text_items][BQ][D] normalised partial outputs
     float* part_lse;    // [n_text_items][BQ] log2-sum-exp of each partial row
     int n_text_items;   // heads * nbt * nsplit
@@ -106,6 +109,7 @@ struct Params {
 struct Item {
     int h, i, e0, n;
     bool split;
+    bool skip;          // head masked out: no work, no output
 };
 
 __device__ inline Item decode_item(const Params& P, int item) {
@@ -125,8 +129,13 @@ __device__ inline Item decode_item(const Params& P, int item) {
         it.i = v - it.h * g.nbv;
         it.e0 = 0;
     }
-    const int c = P.cnt[(size_t)it.h * g.nb + it.i];
-    if (c < 1 || c > g.nb) it.n = -1;   // invalid count: flagged by the softmax role
+    it.skip = P.head_mask != nullptr && P.head_mask[it.h] == 0;
+    if (it.skip) {
+        it.n = 0;
+        return it;
+    }
+    const int c = P.cnt != nullptr ? P.cnt[(size_t)it.h * g.nb + it.i] : g.nb;
+    if (c < 1 || c > g.nb) it.n = -1;   // invalid count: flagged by the epilogue
     else it.n = it.split ? max(0, min(c, it.e0 + kTextChunk) - it.e0) : c;
     return it;
 }
@@ -327,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
     const int first_item = blockIdx.x, stride = gridDim.x;
 
     auto kept_block = [&](const Item& it, int j) -> int {
+        if (P.idx == nullptr) return it.e0 + j;
         int kb = P.idx[((size_t)it.h * nb + it.i) * nb + it.e0 + j];
         if (kb < 0 || kb >= nb) { raise_error(BSA_ERR_DEVICE_ARG); kb = 0; }
         return kb;
@@ -584,7 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             if (next_item < P.n_items) nxt = decode_item(P, next_item);   // prefetched
             const size_t head_off = (size_t)it.h * g.N * D;
             const int q_token = (r < g.B) ? __ldg(P.perm + it.i * g.B + r) : -1;
-            if (it.n <= 0) {
+            if (it.skip) {
+                // head masked out: nothing to write
+            } else if (it.n <= 0) {
                 // nothing kept (an empty text chunk, or an invalid count): zero output
                 if (it.n < 0 && r == 0) raise_error(BSA_ERR_DEVICE_ARG);
                 if (it.split) {
@@ -594,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 } else if (q_token >= 0) {
                     bsa_bf16* orow = P.O + head_off + (size_t)q_token * D;
                     for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                    if (P.lse != nullptr) P.lse[(size_t)it.h * g.N + q_token] = -INFINITY;
                 }
             } else {
                 const int ob = k & 1;
@@ -624,6 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                     }
                     P.part_lse[(size_t)item * BQ + r] = m + __log2f(l);
                 } else {
+                    if (P.lse != nullptr && q_token >= 0) P.lse[(size_t)it.h * g.N + q_token] = m + __log2f(l);
                     // 64 columns at a time: the warp's 32 rows go through a 128B-swizzled staging
                     // tile in shared memory so that each global store instruction writes four
                     // whole 128-byte row segments
@@ -687,6 +701,7 @@ __global__ void merge_text_kernel(Params P) {
     const int h = hr / g.nbt, ti = hr - h * g.nbt;
     const int i = g.nbv + ti;
     if (r >= g.B) return;
+    if (P.head_mask != nullptr && P.head_mask[h] == 0) return;
     const int tok = P.perm[i * g.B + r];
     if (tok < 0) return;
     const int first = (h * g.nbt + ti) * P.nsplit;
@@ -702,6 +717,8 @@ __global__ void merge_text_kernel(Params P) {
     }
     const float o = wsum > 0.f ? acc / wsum : 0.f;
     P.O[(size_t)h * g.N * D + (size_t)tok * D + threadIdx.x] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    if (P.lse != nullptr && threadIdx.x == 0)
+        P.lse[(size_t)h * g.N + tok] = wsum > 0.f ? mx + log2f(wsum) : -INFINITY;
 }
 
 }  // namespace attn

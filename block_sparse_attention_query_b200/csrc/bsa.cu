@@ -14,6 +14,8 @@
 #include "select.cuh"
 #include "drift.cuh"
 #include "attention.cuh"
+#include "mass.cuh"
+#include "correct.cuh"
 
 using namespace bsa;
 
@@ -188,6 +190,13 @@ size_t attention_ws_bytes(const Geom& g) {
     return bytes;
 }
 
+// Captured-mass workspace: [attention workspace][O scratch: heads*N*d bf16]
+// [kept-set lse: heads*N fp32][all-blocks lse: heads*N fp32]
+size_t mass_ws_bytes(const Geom& g) {
+    const size_t rows = (size_t)g.heads * g.N;
+    return attention_ws_bytes(g) + align256(rows * g.d * 2) + 2 * align256(rows * sizeof(float));
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -221,6 +230,39 @@ int launch_attention(const attn::Params& P, cudaStream_t st) {
     return rc;
 }
 
+attn::Params attention_params(const Geom& g, const bsa_bf16* Q, const bsa_bf16* K, const bsa_bf16* V,
+                              const int* idx, const int* cnt, bsa_bf16* O, float* lse, void* ws) {
+    attn::Params P;
+    P.g = g;
+    P.Q = Q;
+    P.K = K;
+    P.V = V;
+    P.idx = idx;
+    P.cnt = cnt;
+    P.O = O;
+    P.lse = lse;
+    P.head_mask = nullptr;
+    P.nsplit = g.nbt > 0 ? text_splits(g) : 1;
+    P.n_text_items = g.heads * g.nbt * (g.nbt > 0 ? P.nsplit : 0);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    P.perm = reinterpret_cast<int*>(w);
+    P.part_o = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g)) : nullptr;
+    P.part_lse = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g) +
+                                                      align256((size_t)P.n_text_items * attn::BQ * g.d * sizeof(float)))
+                           : nullptr;
+    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+    P.n_items = P.n_text_items + g.heads * g.nbv;
+    return P;
+}
+
+int run_attention(const attn::Params& P, cudaStream_t st) {
+    const Geom& g = P.g;
+    if (g.d == 128 && g.B == 128) return launch_attention<128, 128>(P, st);
+    if (g.d == 128) return launch_attention<128, 64>(P, st);
+    if (g.B == 128) return launch_attention<64, 128>(P, st);
+    return launch_attention<64, 64>(P, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -242,6 +284,7 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.score_workspace_bytes = score_ws_bytes(g, prob->score_mode);
     info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
     info.attention_workspace_bytes = attention_ws_bytes(g);
+    info.mass_workspace_bytes = mass_ws_bytes(g);
     *out = info;
     return BSA_OK;
 }
@@ -383,36 +426,64 @@ int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     Geom g;
     const int rc = make_geom(prob, &g);
     if (rc != BSA_OK) return rc;
-    if (Q == nullptr || K == nullptr || V == nullptr || idx == nullptr || cnt == nullptr || O == nullptr)
-        return BSA_ERR_ARG;
+    if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr) return BSA_ERR_ARG;
+    if ((idx == nullptr) != (cnt == nullptr)) return BSA_ERR_ARG;   // both NULL: dense
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(cnt) || !aligned16(O))
         return BSA_ERR_ALIGN;
     const size_t need = attention_ws_bytes(g);
     if (ws == nullptr || ws_bytes < need) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
-    attn::Params P;
-    P.g = g;
-    P.Q = Q;
-    P.K = K;
-    P.V = V;
-    P.idx = idx;
-    P.cnt = cnt;
-    P.O = O;
-    P.nsplit = g.nbt > 0 ? text_splits(g) : 1;
-    P.n_text_items = g.heads * g.nbt * (g.nbt > 0 ? P.nsplit : 0);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    P.perm = reinterpret_cast<int*>(w);
-    P.part_o = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g)) : nullptr;
-    P.part_lse = g.nbt > 0 ? reinterpret_cast<float*>(w + perm_bytes(g) +
-                                                      align256((size_t)P.n_text_items * attn::BQ * g.d * sizeof(float)))
-                           : nullptr;
-    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
-    P.n_items = P.n_text_items + g.heads * g.nbv;
+    const attn::Params P = attention_params(g, Q, K, V, idx, cnt, O, nullptr, ws);
+    return run_attention(P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_dense_correction(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                         const bsa_bf16* V, const int* refresh, bsa_bf16* O, bsa_bf16* R,
+                         void* ws, size_t ws_bytes, bsa_stream_t stream) {
+    Geom g;
+    int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || V == nullptr || refresh == nullptr || O == nullptr || R == nullptr)
+        return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(refresh) || !aligned16(O) || !aligned16(R))
+        return BSA_ERR_ALIGN;
+    if (ws == nullptr || ws_bytes < attention_ws_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (g.d == 128 && g.B == 128) return launch_attention<128, 128>(P, st);
-    if (g.d == 128) return launch_attention<128, 64>(P, st);
-    if (g.B == 128) return launch_attention<64, 128>(P, st);
-    return launch_attention<64, 64>(P, st);
+    // dense attention of the refreshed heads, written into their rows of R
+    attn::Params P = attention_params(g, Q, K, V, nullptr, nullptr, R, nullptr, ws);
+    P.head_mask = refresh;
+    if ((rc = run_attention(P, st)) != BSA_OK) return rc;
+    const long long elems = (long long)g.N * g.d;
+    const dim3 grid((unsigned)((elems + kCorrChunkElems - 1) / kCorrChunkElems), g.heads);
+    correct_kernel<<<grid, kCorrThreads, 0, st>>>(refresh, elems, O, R);
+    return launch_status();
+}
+
+int bsa_captured_mass(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K, const int* idx,
+                      const int* cnt, float* mass, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+    Geom g;
+    int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || idx == nullptr || cnt == nullptr || mass == nullptr) return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(idx) || !aligned16(cnt) || !aligned16(mass))
+        return BSA_ERR_ALIGN;
+    if (ws == nullptr || ws_bytes < mass_ws_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t rows = (size_t)g.heads * g.N;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    bsa_bf16* o_scratch = reinterpret_cast<bsa_bf16*>(w + attention_ws_bytes(g));
+    float* lse_kept = reinterpret_cast<float*>(w + attention_ws_bytes(g) + align256(rows * g.d * 2));
+    float* lse_all = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lse_kept) + align256(rows * sizeof(float)));
+    // the log-sum-exp over the kept keys, then over every key; the outputs themselves are not
+    // needed, so K stands in for V
+    attn::Params P = attention_params(g, Q, K, K, idx, cnt, o_scratch, lse_kept, ws);
+    if ((rc = run_attention(P, st)) != BSA_OK) return rc;
+    P = attention_params(g, Q, K, K, nullptr, nullptr, o_scratch, lse_all, ws);
+    if ((rc = run_attention(P, st)) != BSA_OK) return rc;
+    mass_kernel<<<dim3(g.nb, g.heads), kMassThreads, 0, st>>>(g, P.perm, lse_kept, lse_all, mass);
+    return launch_status();
 }
 
 }  // extern "C"

@@ -7,7 +7,7 @@
 // Float32-grade logits from bf16 tensor cores: both pooled operands (float32) are split into
 // three bf16 parts x = hi + mid + lo (hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid);
 // 24 significant bits), and the six part products down to relative order 2^-16
-//   hi.hi + hi.mid + mid.hi + hi.lo + lo.hi + mid.mid
+//   mid.mid + lo.hi + hi.lo + mid.hi + hi.mid + hi.hi     (issued in this order)
 // accumulate in fp32 TMEM; the dropped terms are of order 2^-24 of the logit, the size of a
 // float32 rounding.
 //
@@ -56,9 +56,12 @@ struct Cfg {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// The six (query part, key part) products, largest first.
-__device__ constexpr int kProdA[6] = {0, 0, 1, 0, 2, 1};
-__device__ constexpr int kProdB[6] = {0, 1, 0, 2, 0, 1};
+// The six (query part, key part) products, SMALLEST first: the tensor cores round the fp32
+// accumulator at every K step, so each step costs up to an ulp of the accumulator's current
+// size. Accumulating the correction products while the sum is still small, and the large
+// hi.hi product last, leaves only hi.hi's own K steps at full size.
+__device__ constexpr int kProdA[6] = {1, 2, 0, 1, 0, 0};
+__device__ constexpr int kProdB[6] = {1, 0, 2, 0, 1, 0};
 
 struct Params {
     Geom g;

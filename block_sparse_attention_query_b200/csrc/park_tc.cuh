@@ -8,7 +8,8 @@
 // Float32-grade logits from bf16 tensor cores: Q is exact in bf16, and each pooled key
 // kbar (float32) is split into three bf16 parts hi + mid + lo (hi = bf16(kbar), mid =
 // bf16(kbar - hi), lo = bf16(kbar - hi - mid); 24 significant bits), so
-// q . kbar = q . hi + q . mid + q . lo accumulates in fp32 TMEM from three MMAs.
+// q . kbar = q . lo + q . mid + q . hi accumulates in fp32 TMEM from three MMAs, smallest
+// first (the tensor cores round the accumulator at every K step, at its current size).
 //
 // Persistent kernel, one CTA per SM, work item = (head, query block). Key blocks come in
 // tiles of 64 (one MMA N). Two passes over the tiles of an item:
@@ -205,14 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t qbase = sQ + qb * C::Q_BYTES;
+                    // lo, then mid, then hi: the small products accumulate while the sum is
+                    // small (each K step rounds the fp32 accumulator at its current size)
 #pragma unroll
-                    for (int sp = 0; sp < 3; ++sp) {
+                    for (int sp = 2; sp >= 0; --sp) {
                         const uint32_t kbase = sK + s * C::STAGE_BYTES + sp * C::KT_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint64_t a = smem_desc_sw128(qbase + (kk >> 2) * C::Q_PANEL + (kk & 3) * 32, 16, 1024);
                             const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * C::KT_PANEL + (kk & 3) * 32, 16, 1024);
-                            mma_bf16_ss(tmem + lb * NT, a, b, C::IDESC, (sp > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16_ss(tmem + lb * NT, a, b, C::IDESC, (sp < 2 || kk > 0) ? 1u : 0u);
                         }
                     }
                     tc_commit(&l_full[lb]);

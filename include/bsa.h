@@ -93,6 +93,7 @@ typedef struct bsa_plan_info {
     size_t score_workspace_bytes;      /* bsa_score_blocks */
     size_t drift_workspace_bytes;      /* bsa_drift_check */
     size_t attention_workspace_bytes;  /* bsa_sparse_attention */
+    size_t mass_workspace_bytes;       /* bsa_captured_mass */
 } bsa_plan_info;
 
 /* Validate `prob` and fill `out`. Host only; launches nothing.
@@ -180,7 +181,9 @@ int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bs
  *   Q, K, V    [heads, tokens, d] bf16, raster order.
  *   idx, cnt   as written by bsa_select_topp (any lists with 1 <= cnt <= nb and distinct
  *              indices in [0, nb) are accepted; a bad entry sets BSA_ERR_DEVICE_ARG in the
- *              device error word and the row's output is unspecified).
+ *              device error word and the row's output is unspecified). Both NULL: every
+ *              block is kept (dense attention, e.g. the steps before a one-shot estimate, or a
+ *              dense refresh); only one NULL is BSA_ERR_ARG.
  *   O          [heads, tokens, d] bf16 out, raster order. Every real token is written.
  *   ws         at least plan.attention_workspace_bytes, always required: the block-slot ->
  *              token table, and the partial results of the dense text rows, which are split
@@ -188,6 +191,42 @@ int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bs
 int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                          const bsa_bf16* V, const int* idx, const int* cnt, bsa_bf16* O,
                          void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Cached dense correction of this step's sparse output (RECAP: Reciprocal Sparse Attention
+ * and Hierarchical Caching for Efficient Video Diffusion, Abstract: a cached dense refinement
+ * corrects the interactions the current sparse estimate omits, and fresh statistics of the
+ * inputs regulate the aging correction). Call after bsa_sparse_attention of the same step,
+ * with the refresh flags of bsa_drift_check (the fresh statistics):
+ *   refresh[h] != 0: D = dense attention of head h (every key block); R_h = D - O_h (the new
+ *                    correction); O_h = D.
+ *   refresh[h] == 0: O_h = O_h + R_h (the sparse output plus the head's cached correction).
+ * bf16 in and out, float32 arithmetic.
+ *   Q, K, V    [heads, tokens, d] bf16, raster order (this step's).
+ *   refresh    [heads] int, device (from bsa_drift_check; all 1 on the first step).
+ *   O          [heads, tokens, d] bf16 in/out: this step's sparse output in, corrected out.
+ *   R          [heads, tokens, d] bf16 in/out: the cached corrections, caller-owned across
+ *              steps; its contents only matter for heads that are not refreshed.
+ *   ws         at least plan.attention_workspace_bytes. */
+int bsa_dense_correction(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                         const bsa_bf16* V, const int* refresh, bsa_bf16* O, bsa_bf16* R,
+                         void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Retrieval accuracy of a set of kept-block lists (PARK, Abstract: inaccurate block
+ * retrieval either degrades quality or wastes computation; retrieval is judged by its
+ * accuracy). For every real query t of query block i of head h, the captured mass is the
+ * share of t's exact attention softmax over ALL real keys that falls on the real keys of the
+ * kept blocks idx[h][i][0..cnt[h][i]-1]; mass[h][i] is its mean over the block's real
+ * queries (1 when every block is kept). A measurement, not a step of the hot path: it runs
+ * the attention kernel twice (kept blocks, then every block) for the two log-sum-exps of
+ * each query and takes 2^(difference), so it costs one dense attention pass.
+ *   Q, K       [heads, tokens, d] bf16, raster order.
+ *   idx, cnt   kept lists as bsa_select_topp writes them (same checks as bsa_sparse_attention).
+ *   mass       [heads, nb] float32 out.
+ *   ws         at least plan.mass_workspace_bytes: the attention workspace, an output scratch
+ *              [heads, tokens, d] bf16 and two [heads, tokens] float32 log-sum-exps. */
+int bsa_captured_mass(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
+                      const int* idx, const int* cnt, float* mass,
+                      void* ws, size_t ws_bytes, bsa_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the current device.
  * Returns BSA_OK, BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_ARG or BSA_ERR_CUDA. */

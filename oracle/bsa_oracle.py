@@ -20,6 +20,8 @@ the slow, obvious way, in the order the pages describe the method:
    attention mass that falls on its kept key blocks
 9. ``rapid_run``       — one-shot block-importance estimate early in the run, cached scores
    and mask reused for the later steps, optional staged re-selection (Turbo)
+10. ``recap_run``      — sparse attention corrected by a cached dense residual, refreshed
+   per head when its query-key drift says the correction has aged
 
 Sources (page title, then the part of the page):
 * PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers —
@@ -35,6 +37,10 @@ Sources (page title, then the part of the page):
 * RAPID: Reusing Attention Sparsity with Inter-step Adaptation for Efficient Video
   Diffusion — English abstract: 3D attention, block importance estimated and the sparse
   mask cached for reuse across steps.
+* RECAP: Reciprocal Sparse Attention and Hierarchical Caching for Efficient Video Diffusion
+  — Abstract: a cached dense refinement corrects the interactions the current sparse
+  estimate omits, and fresh sparse statistics track the inputs and regulate the aging
+  correction.
 * PARK — Abstract: inaccurate block retrieval either degrades quality or wastes computation;
   PARK is judged by its block retrieval accuracy (``captured_mass`` measures it without a
   model: how much of the exact attention the retrieved blocks hold).
@@ -435,4 +441,59 @@ def rapid_run(steps_qk, V, layout, p0, estimate_step=0, stages=(), mode="meanpoo
             out["O"].append(np.stack(Os))
     out["masks"] = masks
     out["scores"] = scores
+    return out
+
+
+# ------------------------------------------------------------ 10. cached dense correction
+
+def dense_attention_head(Qh, Kh, Vh, layout: Layout) -> np.ndarray:
+    """Attention over every key block (the kept list of every row is all blocks)."""
+    idx = np.tile(np.arange(layout.nb, dtype=np.int32), (layout.nb, 1))
+    cnt = np.full(layout.nb, layout.nb, dtype=np.int32)
+    return sparse_attention_head(Qh, Kh, Vh, idx, cnt, layout)
+
+
+def recap_run(steps_qk, V, layout, p, tau, mode="meanpool"):
+    """Sparse attention with a cached dense correction, refreshed per head on drift.
+
+    RECAP abstract: a cached dense refinement corrects the interactions that the current
+    sparse estimate omits, while fresh sparse statistics follow the input changes and
+    regulate the aging correction. Readings (the abstract gives no formula; the rest of RECAP,
+    whole-step prediction reuse and its error feedback, is out of scope here):
+    * the correction of head h is R_h = O_dense - O_sparse at the head's last refresh step;
+    * the fresh statistics are the per-head query-key drift of Temporal Mask Reuse (HEART
+      abstract): a head whose drift since its last refresh exceeds tau (or that has no cache
+      yet) refreshes its mask, its dense output and its correction, and outputs the dense
+      attention; every other head outputs its current sparse attention plus its cached R.
+
+    `steps_qk` yields (Q, K) bf16 bits [heads, N, d] per step; V is fixed. Returns per-step
+    refresh flags, outputs and the final corrections.
+    """
+    heads = V.shape[0]
+    Vf = [bf16_to_f64(V[h]) for h in range(heads)]
+    ref = [None] * heads
+    masks = [None] * heads
+    corr = [None] * heads
+    out = {"refresh": [], "O": []}
+    for Q, K in steps_qk:
+        flags, Os = [], []
+        for h in range(heads):
+            Qh, Kh = bf16_to_f64(Q[h]), bf16_to_f64(K[h])
+            delta = math.inf if ref[h] is None else drift(Qh, Kh, ref[h][0], ref[h][1])
+            fresh = refresh_decision(delta, tau, ref[h] is not None)
+            if fresh:
+                S = score_head(Qh, Kh, layout, mode).astype(np.float32)
+                masks[h] = select_topp(S, p[h], layout)
+                ref[h] = (Qh, Kh)
+            O_sparse = sparse_attention_head(Qh, Kh, Vf[h], masks[h][0], masks[h][1], layout)
+            if fresh:
+                O_dense = dense_attention_head(Qh, Kh, Vf[h], layout)
+                corr[h] = O_dense - O_sparse
+                Os.append(O_dense)
+            else:
+                Os.append(O_sparse + corr[h])
+            flags.append(fresh)
+        out["refresh"].append(flags)
+        out["O"].append(np.stack(Os))
+    out["R"] = corr
     return out

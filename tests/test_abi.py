@@ -21,12 +21,12 @@ from tests.conftest import GOLDEN, ROOT  # noqa: E402
 def _declared_symbols():
     with open(os.path.join(ROOT, "include", "bsa.h")) as f:
         text = f.read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(bsa_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^(?:const\s+)?(?:unsigned\s+)?(?:long\s+)*\w+\s*\*?\s*(bsa_\w+)\s*\(", text, re.M)))
 
 
 def test_exports_every_declared_symbol():
     names = _declared_symbols()
-    assert "bsa_sparse_attention" in names and len(names) >= 9
+    assert "bsa_sparse_attention" in names and "bsa_launch_count" in names and len(names) >= 12
     for n in names:
         assert hasattr(bsa.lib, n), n
         assert n in bsa.EXPORTS, n
@@ -84,6 +84,7 @@ def test_plan_rejects_bad_problems():
 
 def test_calls_reject_bad_pointers_before_launch():
     # host-side validation only: no pointer is dereferenced and nothing is launched
+    launches_before = bsa.bsa_launch_count()
     prob = bsa.problem(2, 64, 4, 16, 16, 0, 64)
     L = bsa.lib
     a = ctypes.c_void_p(4096)          # aligned, never dereferenced on these paths
@@ -100,9 +101,23 @@ def test_calls_reject_bad_pointers_before_launch():
     assert L.bsa_drift_check(pr, a, a, a, a, ctypes.c_float(0.05), 0, a, a, a, 8, None) == bsa.BSA_ERR_WORKSPACE
     assert L.bsa_drift_check(pr, a, a, a, None, ctypes.c_float(0.05), 0, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG
     assert L.bsa_sparse_attention(pr, a, a, a, a, a, None, a, 1 << 20, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_sparse_attention(pr, a, a, a, None, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG   # idx alone NULL
+    assert L.bsa_sparse_attention(pr, a, a, a, a, None, a, a, 1 << 20, None) == bsa.BSA_ERR_ARG   # cnt alone NULL
     assert L.bsa_sparse_attention(pr, a, a, mis, a, a, a, a, 1 << 20, None) == bsa.BSA_ERR_ALIGN
     assert L.bsa_sparse_attention(pr, a, a, a, a, a, a, None, 1 << 20, None) == bsa.BSA_ERR_WORKSPACE
     text = bsa.problem(2, 64, 4, 16, 16, 64, 64)
     need = bsa.bsa_plan(text).attention_workspace_bytes
     assert need > 0
     assert L.bsa_sparse_attention(ctypes.byref(text), a, a, a, a, a, a, a, need - 1, None) == bsa.BSA_ERR_WORKSPACE
+    # captured mass: the same host checks, and a workspace of plan.mass_workspace_bytes
+    need = bsa.bsa_plan(prob).mass_workspace_bytes
+    assert need > bsa.bsa_plan(prob).attention_workspace_bytes
+    assert L.bsa_captured_mass(pr, a, a, a, a, None, a, need, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_captured_mass(pr, a, mis, a, a, a, a, need, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_captured_mass(pr, a, a, a, a, a, a, need - 1, None) == bsa.BSA_ERR_WORKSPACE
+    # dense correction: pointers, alignment, workspace
+    aw = bsa.bsa_plan(prob).attention_workspace_bytes
+    assert L.bsa_dense_correction(pr, a, a, a, None, a, a, a, aw, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_dense_correction(pr, a, a, a, a, a, mis, a, aw, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_dense_correction(pr, a, a, a, a, a, a, a, aw - 1, None) == bsa.BSA_ERR_WORKSPACE
+    assert bsa.bsa_launch_count() == launches_before     # none of the rejected calls launched

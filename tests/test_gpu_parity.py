@@ -426,3 +426,182 @@ def test_select_flat_and_peaked_rows(conc, p):
     assert res["window"] <= PT.exempt_limit(res["rows"]), res
     if conc >= 5.0:
         assert cnt.cpu().numpy().mean() > 64       # the fallback path was exercised
+
+
+# ------------------------------------------------------------------ retrieval accuracy
+# Tolerance of the captured mass 2^(lse_kept - lse_all): each log-sum-exp carries the float32
+# error of its logits (<= 4u * sum_c |q_c k_c| / sqrt(d), about 3e-5 for these inputs) and of
+# its sum of up to N exponentials (relative (4 sqrt(n) + 32)u, about 1e-4 at n = 119k); the
+# difference of two, through 2^x, stays under 2e-4 of a mass that is at most 1.
+MASS_ATOL = 2e-4
+
+
+def _gpu_mass(c, idx, cnt):
+    bsa = _bsa()
+    mass = torch.full((c.heads, c.nb), float("nan"), dtype=torch.float32, device="cuda")
+    bsa.bsa_captured_mass(c.prob, c.Q, c.K, idx, cnt, mass, c.ws(c.plan.mass_workspace_bytes))
+    _status_ok()
+    return mass.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("mode", ["meanpool", "park"])
+def test_captured_mass_matches_oracle(name, mode):
+    c = Case(**SMALL[name], mode=mode)
+    idx, cnt = _oracle_mask(c)
+    got = _gpu_mass(c, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    for h in range(c.heads):
+        ref = O.captured_mass(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]), idx[h], cnt[h], c.layout)
+        err = np.abs(got[h] - ref)
+        assert err.max() <= MASS_ATOL, (name, mode, h, float(err.max()))
+    # text rows keep every block: all of the mass
+    if c.layout.nb_text:
+        assert np.allclose(got[:, c.layout.nb_video:], 1.0, atol=MASS_ATOL)
+
+
+def test_captured_mass_all_blocks_is_one():
+    c = Case(**SMALL["text_d128_b128"])
+    idx = np.tile(np.arange(c.nb, dtype=np.int32), (c.heads, c.nb, 1))
+    cnt = np.full((c.heads, c.nb), c.nb, np.int32)
+    got = _gpu_mass(c, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    assert np.abs(got - 1.0).max() <= MASS_ATOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["wan13b_480p", "hunyuan_720p"])
+def test_full_size_captured_mass_sampled(name):
+    # the GPU's masks at full size; sampled query blocks (the last one, text rows included)
+    # against the oracle's dense softmax
+    c = _full_case(name)
+    idx, cnt = c.gpu_select(c.gpu_scores())
+    got = _gpu_mass(c, idx, cnt)
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    rng = np.random.default_rng(1)
+    for h in (0, c.heads - 1):
+        qbl = sorted(set(rng.choice(c.layout.nb, 4, replace=False).tolist() + [c.layout.nb - 1]))
+        ref = O.captured_mass(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]), idx_h[h], cnt_h[h], c.layout,
+                              qblocks=qbl)
+        err = np.abs(got[h, qbl] - ref[qbl])
+        assert err.max() <= MASS_ATOL, (name, h, float(err.max()))
+    assert np.isfinite(got).all() and got.min() > 0 and got.max() <= 1 + MASS_ATOL
+
+
+# ------------------------------------------------------------------ one-shot schedule
+
+def test_one_shot_turbo_schedule_follows_oracle():
+    """Dense steps, the one-shot estimate, reuse and two Turbo stages on the tiny random walk:
+    what each step did, the kept lists and the outputs follow the oracle step by step."""
+    from block_sparse_attention_query_b200.layer import OneShotLayer
+    w = inputs.workload("tiny")
+    walk = inputs.RandomWalk(w.heads, w.d, w.T, w.H, w.W, 0, seed=1)
+    stages = [(5, 0.8), (8, 0.7)]
+    layer = OneShotLayer(w.heads, w.d, w.T, w.H, w.W, 0, w.block, p=0.95, estimate_step=2, stages=stages)
+    L = O.block_layout(w.T, w.H, w.W, 0, w.block)
+    Vd = PT.to_dev_bf16(walk.V)
+    Od = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device="cuda")
+    steps, kinds, cnts, outs = [], [], [], []
+    for s in range(10):
+        q, k, _ = walk.current()
+        steps.append((q, k))
+        layer.step(PT.to_dev_bf16(q), PT.to_dev_bf16(k), Vd, Od)
+        kinds.append(layer.kind)
+        cnts.append(layer.cnt.cpu().numpy().copy())
+        outs.append(PT.bf16_bits_f64(PT.from_dev_bf16(Od)))
+        walk.advance()
+    _status_ok()
+    ref = O.rapid_run(steps, walk.V, L, [0.95] * w.heads, estimate_step=2, stages=stages)
+    assert kinds == ref["kind"]
+    S = layer.scores.cpu().numpy()
+    for h in range(w.heads):
+        # the cached scores are those of the estimate step
+        Qh, Kh = O.bf16_to_f64(steps[2][0][h]), O.bf16_to_f64(steps[2][1][h])
+        Sx = O.score_meanpool(Qh, Kh, L)
+        _check_scores(S[h], Sx, PT.score_bound(Qh, Kh, L, "meanpool", Sx), ("one-shot", h))
+    for s in range(10):
+        if ref["kind"][s] != "dense":
+            assert all(np.array_equal(cnts[s][h], ref["cnt"][s][h]) for h in range(w.heads)), s
+        mx, rel = PT.attention_errors(outs[s], ref["O"][s], np.arange(w.tokens))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (s, ref["kind"][s], mx, rel)
+    # the stages pruned: fewer kept blocks at the end than at the estimate
+    assert cnts[9].sum() < cnts[2].sum()
+
+
+def test_dense_attention_without_lists():
+    # idx = cnt = NULL keeps every block: dense softmax attention
+    c = Case(**SMALL["text_d64_b128"])
+    bsa = _bsa()
+    Od = torch.full((c.heads, c.N, c.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bsa.bsa_sparse_attention(c.prob, c.Q, c.K, c.V, None, None, Od, c.ws(c.plan.attention_workspace_bytes))
+    _status_ok()
+    got = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    for h in range(c.heads):
+        q, k, v = (torch.from_numpy(O.bf16_to_f64(x[h])) for x in (c.Qb, c.Kb, c.Vb))
+        ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0].numpy()
+        mx, rel = PT.attention_errors(got[h], ref, np.arange(c.N))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (h, mx, rel)
+
+
+# --------------------------------------------------------------- cached dense correction
+
+def test_dense_correction_follows_oracle():
+    """Drift-gated sparse attention with a cached dense correction over 40 steps of the tiny
+    random walk (refreshes at step 0 and again when the drift passes tau): refresh flags and
+    outputs follow the oracle step by step. The correction is stored in bf16, so outputs are
+    held to the attention tolerance."""
+    from block_sparse_attention_query_b200.layer import CorrectedLayer
+    w = inputs.workload("tiny")
+    walk = inputs.RandomWalk(w.heads, w.d, w.T, w.H, w.W, 0, seed=2)
+    layer = CorrectedLayer(w.heads, w.d, w.T, w.H, w.W, 0, w.block, p=0.8, tau=0.05)
+    L = O.block_layout(w.T, w.H, w.W, 0, w.block)
+    Vd = PT.to_dev_bf16(walk.V)
+    Od = torch.empty(w.heads, w.tokens, w.d, dtype=torch.bfloat16, device="cuda")
+    steps, flags, outs = [], [], {}
+    check = (0, 1, 20, 39)
+    for s in range(40):
+        q, k, _ = walk.current()
+        steps.append((q, k))
+        layer.step(PT.to_dev_bf16(q), PT.to_dev_bf16(k), Vd, Od)
+        flags.append(layer.refresh.cpu().tolist())
+        if s in check:
+            outs[s] = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+        walk.advance()
+    _status_ok()
+    ref = O.recap_run(steps, walk.V, L, [0.8] * w.heads, 0.05)
+    flags_ref = [[int(x) for x in f] for f in ref["refresh"]]
+    assert flags == flags_ref
+    assert sum(map(sum, flags_ref)) > w.heads          # a second refresh happened
+    for s in check:
+        mx, rel = PT.attention_errors(outs[s], ref["O"][s], np.arange(w.tokens))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (s, mx, rel)
+    # the cached correction itself (bf16) against the oracle's
+    R = PT.bf16_bits_f64(PT.from_dev_bf16(layer.R))
+    for h in range(w.heads):
+        mx = float(np.abs(R[h] - ref["R"][h]).max())
+        assert mx <= ATT_MAX_ABS, (h, mx)
+
+
+def test_dense_correction_heads_masked():
+    # refresh only head 1: head 0 gets O + R, head 1 the dense output and a new R
+    c = Case(**SMALL["text_d64_b128"])
+    bsa = _bsa()
+    idx, cnt = _oracle_mask(c)
+    Od = c.gpu_attention(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda())
+    sparse = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    rng = np.random.default_rng(3)
+    R0 = inputs.f32_to_bf16_bits((rng.standard_normal((c.heads, c.N, c.d)) * 0.01).astype(np.float32))
+    Rd = PT.to_dev_bf16(R0)
+    refresh = torch.tensor([0, 1, 0], dtype=torch.int32, device="cuda")
+    bsa.bsa_dense_correction(c.prob, c.Q, c.K, c.V, refresh, Od, Rd, c.ws(c.plan.attention_workspace_bytes))
+    _status_ok()
+    out = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    Rn = PT.bf16_bits_f64(PT.from_dev_bf16(Rd))
+    R0f = O.bf16_to_f64(R0)
+    for h in (0, 2):
+        expect = inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits((sparse[h] + R0f[h]).astype(np.float32)))
+        assert np.array_equal(out[h], expect.astype(np.float64))
+        assert np.array_equal(Rn[h], R0f[h])
+    q, k, v = (torch.from_numpy(O.bf16_to_f64(x[1])) for x in (c.Qb, c.Kb, c.Vb))
+    dense = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0].numpy()
+    mx, rel = PT.attention_errors(out[1], dense, np.arange(c.N))
+    assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2
+    assert np.abs(Rn[1] - (out[1] - sparse[1])).max() <= 2 ** -8 * np.abs(out[1] - sparse[1]).max() + 1e-6

@@ -419,3 +419,41 @@ def test_rapid_turbo_stages_prune_the_cached_ranking():
         for i in range(L.nb):
             order = O.sort_row(S[i])
             assert list(r["masks"][h][0][i, :cnt[i]]) == [int(j) for j in order[:cnt[i]]]
+
+
+# ------------------------------------------------------------ cached dense correction
+
+def test_recap_static_inputs_reproduce_dense_attention_every_step():
+    # without drift the sparse output never changes, so sparse + cached correction is exactly
+    # the dense attention of the refresh step, at every step
+    steps, V, L = _walk_steps(1)
+    steps = steps * 4
+    r = O.recap_run(steps, V, L, [0.7, 0.7], tau=0.05)
+    assert [list(f) for f in r["refresh"]] == [[True, True]] + [[False, False]] * 3
+    for h in range(V.shape[0]):
+        q, k, v = (torch.from_numpy(O.bf16_to_f64(x[h])) for x in (steps[0][0], steps[0][1], V))
+        dense = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0].numpy()
+        for s in range(4):
+            assert np.allclose(r["O"][s][h], dense, atol=1e-12)
+        assert np.abs(r["R"][h]).max() > 1e-3        # the correction is not trivial at p = 0.7
+
+
+def test_recap_correction_is_zero_when_every_block_is_kept():
+    steps, V, L = _walk_steps(3)
+    r = O.recap_run(steps, V, L, [1.0, 1.0], tau=0.05)
+    for h in range(V.shape[0]):
+        assert np.abs(r["R"][h]).max() < 1e-12
+
+
+def test_recap_between_refreshes_is_sparse_plus_cached_residual():
+    steps, V, L = _walk_steps(4)
+    r = O.recap_run(steps, V, L, [0.7, 0.7], tau=10.0)   # never refreshes after step 0
+    for h in range(V.shape[0]):
+        Q0, K0 = O.bf16_to_f64(steps[0][0][h]), O.bf16_to_f64(steps[0][1][h])
+        Vh = O.bf16_to_f64(V[h])
+        S = O.score_meanpool(Q0, K0, L).astype(np.float32)
+        idx, cnt = O.select_topp(S, 0.7, L)
+        R0 = O.dense_attention_head(Q0, K0, Vh, L) - O.sparse_attention_head(Q0, K0, Vh, idx, cnt, L)
+        Q3, K3 = O.bf16_to_f64(steps[3][0][h]), O.bf16_to_f64(steps[3][1][h])
+        expect = O.sparse_attention_head(Q3, K3, Vh, idx, cnt, L) + R0
+        assert np.allclose(r["O"][3][h], expect, atol=1e-12)
