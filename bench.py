@@ -21,6 +21,7 @@ slowest rank's time per layer call (strong scaling: the layer is fixed and N GPU
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -171,6 +172,8 @@ def run_ours(args, ws, rank, local):
     from block_sparse_attention_query_b200.layer import SparseAttentionLayer
 
     w = inputs.workload(args.workload)
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads, p=tuple(w.p[:args.heads]))
     h0, h1 = head_range(w.heads, ws, rank)
     Hl = h1 - h0
     B, d, N = w.block, w.d, w.tokens
@@ -293,7 +296,7 @@ def run_ours(args, ws, rank, local):
         b = bytes_drift if dom == "drift_check" else bytes_score
         ach = b * per_gpu / (stage_ms[names.index(dom)] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4)}
-    traffic = args.traffic if args.traffic is not None else (_profiled_traffic(dom, w.name) if ws == 1 else None)
+    traffic = args.traffic if args.traffic is not None else (_profiled_traffic(dom, w.name) if ws == 1 and not args.heads else None)
     roof.update({"kernel": dom,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
                  "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
@@ -339,7 +342,7 @@ def run_ours(args, ws, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded RFF-structured Q/K, Gaussian V; no model weights)",
-        "config": {"workload": w.name, "heads": H, "d": d, "grid": [w.T, w.H, w.W],
+        "config": {"workload": w.name + (f" (first {w.heads} heads)" if args.heads else ""), "heads": H, "d": d, "grid": [w.T, w.H, w.W],
                    "text_tokens": w.text_tokens, "tokens": N, "block": B, "blocks": plan.nb,
                    "top_p": sorted(set(float(x) for x in w.p)), "scorer": args.mode,
                    "parallelism": (f"heads split over {ws} GPUs, {Hl} per GPU, no data-path collective"
@@ -578,6 +581,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--mode", default="meanpool", choices=["meanpool", "park"])
     ap.add_argument("--gather", action="store_true", help="all-gather O over the ranks every step (N > 1)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first H heads of the layer (same shape per head; for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-retrieval", action="store_true", help="skip the retrieval-accuracy measurement")

@@ -17,6 +17,11 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsa.so")
+# Test-only variant: bounded waits of about 10 ms instead of 2 s, and a hook that makes the
+# attention kernel take its timeout path (tests/test_wait_timeout.py). Never loaded by the
+# package itself.
+WAITTEST_LIB = os.path.join(PKG, "libbsa_waittest.so")
+WAITTEST_FLAGS = ["-DBSA_TEST_HOOKS", "-DBSA_WAIT_LIMIT_CYCLES=20000000LL"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,25 +43,37 @@ def _sources():
                   + [os.path.join(ROOT, "include", "bsa.h")])
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
+def _compile(lib: str, extra, verbose: bool) -> str:
     units = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *units]
+    tmp = lib + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", tmp, *units]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not needs_build(LIB):
+        return LIB
+    return _compile(LIB, [], verbose)
+
+
+def build_wait_test(force: bool = False, verbose: bool = False) -> str:
+    """The test-only variant with short waits and the timeout hook."""
+    if not force and not needs_build(WAITTEST_LIB):
+        return WAITTEST_LIB
+    return _compile(WAITTEST_LIB, WAITTEST_FLAGS, verbose)
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_wait_test(force="--force" in sys.argv, verbose=True))

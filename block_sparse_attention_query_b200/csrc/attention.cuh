@@ -260,6 +260,13 @@ __device__ inline void gather_tile(const RowToks<D, ROWS>& rt, const bsa_bf16* h
         cp_async_16(tile_smem + sw128_offset(ROWS, r0 + k, c), head_base + (size_t)rt.t[k] * D + c * 8);
 }
 
+#ifdef BSA_TEST_HOOKS
+// Test builds only (never in the product library): while set, CTA 0 withholds the arrival of
+// its first query tile, so the MMA warp's bounded wait on it runs out and the launch takes
+// the timeout path (BSA_ERR_TIMEOUT, every role winds down, TMEM is freed).
+__device__ int g_test_withhold_q;
+#endif
+
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P) {
     using C = Cfg<D, BK>;
@@ -363,6 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch);
             if (!ok) break;
             gather_tile<D, BQ>(tq, P.Q + head_off, sQ + qb * C::Q_BYTES, lt);
+#ifdef BSA_TEST_HOOKS
+            if (!(k == 0 && blockIdx.x == 0 && *(volatile int*)&g_test_withhold_q != 0))
+#endif
             cp_async_arrive_noinc(&q_full[qb]);
             for (int j = 0; j < it.n && ok; ++j, ++gblk) {
                 const int ks = gblk % NK, vs = gblk % NV;
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             }
             ++k;
         }
-        cp_async_wait<0>();   // no copy may still target shared memory at teardown
+        cp_async_wait_all();   // no copy may still target shared memory at teardown
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issuer
         if (elect_one()) {

@@ -578,4 +578,12 @@ const char* bsa_version(void) { return "bsa 0.2.0 sm_100a"; }
 
 unsigned long long bsa_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 
+#ifdef BSA_TEST_HOOKS
+// Test builds only: makes the next attention launches take their timeout path (see
+// attn::g_test_withhold_q). Not declared in bsa.h and not in the product library.
+int bsa_test_withhold_q_arrival(int on) {
+    return cudaMemcpyToSymbol(attn::g_test_withhold_q, &on, sizeof(int)) == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+#endif
+
 }  // extern "C"

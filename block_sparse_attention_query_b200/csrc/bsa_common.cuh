@@ -177,9 +177,9 @@ __device__ inline uint4 ld_shared_v4(uint32_t addr) {
 __device__ inline void cp_async_16(uint32_t dst_smem, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
-__device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ inline void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Waits until every cp.async this thread has issued has landed, committed to a group or not
+// (the gathers signal through mbarriers and are never committed; wait_group would skip them).
+__device__ inline void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Arrive on `bar` (without raising its expected count) once every cp.async this thread has
 // issued so far has landed in shared memory.

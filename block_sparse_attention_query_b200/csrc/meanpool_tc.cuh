@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             }
             ++k;
         }
-        cp_async_wait<0>();
+        cp_async_wait_all();   // no copy may still target shared memory at teardown
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issuer
         if (elect_one()) {
