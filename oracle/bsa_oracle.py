@@ -22,6 +22,8 @@ the slow, obvious way, in the order the pages describe the method:
    and mask reused for the later steps, optional staged re-selection (Turbo)
 10. ``recap_run``      — sparse attention corrected by a cached dense residual, refreshed
    per head when its query-key drift says the correction has aged
+11. ``cluster_keys``   — PARK's key side: keys grouped by k-means in a metric built from the
+   current queries, so that keys the queries score alike share a key block
 
 Sources (page title, then the part of the page):
 * PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion Transformers —
@@ -497,3 +499,86 @@ def recap_run(steps_qk, V, layout, p, tau, mode="meanpool"):
         out["O"].append(np.stack(Os))
     out["R"] = corr
     return out
+
+
+# ----------------------------------------------------------- 11. query-aware key blocks
+
+def query_metric(Qh: np.ndarray, layout: Layout) -> np.ndarray:
+    """M = (1/n) sum over the head's real queries q of q q^T (d x d).
+
+    For two keys, (k1 - k2)^T M (k1 - k2) is the mean over the queries of (q.k1 - q.k2)^2: how
+    differently the current queries score them. Reading of PARK abstract ("uses information
+    from the current queries to transform keys before clustering, so that keys receiving
+    similar QK scores are grouped together"): the transform is k -> L^T k with M = L L^T, under
+    which Euclidean distance is exactly that score difference; clustering in the transformed
+    space is clustering with the metric M.
+    """
+    rows = np.concatenate([layout.rows(i) for i in range(layout.nb)])
+    Q = Qh[rows]
+    return Q.T @ Q / len(rows)
+
+
+def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2):
+    """Query-aware key blocks (PARK abstract, key-side clustering).
+
+    Readings (the page gives no formula): the video keys are clustered by Lloyd's k-means
+    with the metric M of `query_metric`, into as many clusters as there are video blocks,
+    starting from the means of the 3D-tile blocks; each of `iters` rounds assigns every key
+    to the centroid c_j minimising (k - c_j)^T M (k - c_j) (ties to the lowest j), then moves
+    every non-empty cluster's centroid to the mean of its keys. The key blocks then follow the
+    block rule of the query side: the video keys in order of (cluster, raster index), cut every
+    B keys (so every key block keeps its tile-layout size); text key blocks are unchanged.
+    Returns (key_perm int64 [nb*B] like Layout.perm, assignment int64 [Nv] of the last round).
+    """
+    if iters < 1:
+        raise ValueError("iters >= 1")
+    M = query_metric(Qh, layout)
+    nv = layout.nb_video
+    Nv = int(layout.counts[:nv].sum())
+    Kv = Kh[:Nv]
+    C = np.stack([Kh[layout.rows(j)].mean(axis=0) for j in range(nv)])
+    a = None
+    for _ in range(iters):
+        W = C @ M                                   # w_j = M c_j  (M symmetric)
+        b = (C * W).sum(axis=1)                     # c_j^T M c_j
+        obj = b[None, :] - 2.0 * (Kv @ W.T)         # (k - c_j)^T M (k - c_j) - k^T M k
+        a = np.argmin(obj, axis=1)                  # first index on ties
+        for j in range(nv):
+            members = Kv[a == j]
+            if len(members):
+                C[j] = members.mean(axis=0)
+    order = np.lexsort((np.arange(Nv), a))          # by cluster, then raster index
+    key_perm = layout.perm.copy()
+    key_perm[:Nv] = order
+    return key_perm, a
+
+
+def key_layout(layout: Layout, key_perm: np.ndarray) -> Layout:
+    """The block layout of the key side after `cluster_keys` (same block sizes)."""
+    return Layout(np.asarray(key_perm, dtype=np.int64), layout.B, layout.nb, layout.nb_video,
+                  layout.nb_text, layout.counts.copy())
+
+
+def score_park_keys(Qh, Kh, qlayout: Layout, klayout: Layout) -> np.ndarray:
+    """PARK scores with separate query and key block layouts (key blocks from cluster_keys)."""
+    d = Qh.shape[1]
+    kbar = pool_blocks(Kh, klayout)
+    P = np.zeros((qlayout.nb, klayout.nb), dtype=np.float64)
+    for i in range(qlayout.nb):
+        q = Qh[qlayout.rows(i)]
+        P[i] = _softmax_rows(q @ kbar.T / math.sqrt(d)).mean(axis=0)
+    return P
+
+
+def sparse_attention_keys(Qh, Kh, Vh, idx, cnt, qlayout: Layout, klayout: Layout, qblocks=None):
+    """sparse_attention_head with the key blocks of `klayout` (query blocks of `qlayout`)."""
+    N, d = Qh.shape
+    O = np.full((N, Vh.shape[1]), np.nan, dtype=np.float64)
+    scale = 1.0 / math.sqrt(d)
+    for i in (range(qlayout.nb) if qblocks is None else qblocks):
+        rows = qlayout.rows(i)
+        keys = np.concatenate([klayout.rows(int(j)) for j in idx[i, :cnt[i]]])
+        L = (Qh[rows] @ Kh[keys].T) * scale
+        e = np.exp(L - L.max(axis=1, keepdims=True))
+        O[rows] = (e @ Vh[keys]) / e.sum(axis=1, keepdims=True)
+    return O

@@ -457,3 +457,80 @@ def test_recap_between_refreshes_is_sparse_plus_cached_residual():
         Q3, K3 = O.bf16_to_f64(steps[3][0][h]), O.bf16_to_f64(steps[3][1][h])
         expect = O.sparse_attention_head(Q3, K3, Vh, idx, cnt, L) + R0
         assert np.allclose(r["O"][3][h], expect, atol=1e-12)
+
+
+# --------------------------------------------------------------- query-aware key blocks
+
+def _cluster_case(seed=21, T=2, H=8, W=16, text=24, B=32, tile=(1, 4, 8), d=8):
+    rng = np.random.default_rng(seed)
+    L = O.block_layout(T, H, W, text, B, tile)
+    N = T * H * W + text
+    Q = _bf16_round_f64(rng.standard_normal((N, d)) * np.linspace(0.3, 2.0, d))
+    K = _bf16_round_f64(rng.standard_normal((N, d)))
+    return L, Q, K
+
+
+def test_query_metric_is_mean_square_score_difference():
+    L, Q, K = _cluster_case()
+    M = O.query_metric(Q, L)
+    k1, k2 = K[3], K[77]
+    assert (k1 - k2) @ M @ (k1 - k2) == pytest.approx(np.mean((Q @ k1 - Q @ k2) ** 2), rel=1e-12)
+
+
+def test_cluster_keys_is_kmeans_on_cholesky_transformed_keys():
+    # a library routine on the transformed keys: sklearn's Lloyd k-means, same initial centres
+    from sklearn.cluster import KMeans
+    L, Q, K = _cluster_case()
+    nv = L.nb_video
+    Nv = int(L.counts[:nv].sum())
+    Lc = np.linalg.cholesky(O.query_metric(Q, L))
+    X = K[:Nv] @ Lc                                 # rows are (L^T k)^T
+    init = np.stack([X[L.rows(j)].mean(axis=0) for j in range(nv)])
+    for iters in (1, 2, 3):
+        _, a = O.cluster_keys(Q, K, L, iters)
+        km = KMeans(n_clusters=nv, init=init, n_init=1, max_iter=iters, tol=0.0, algorithm="lloyd").fit(X)
+        # sklearn reports the labels of its last assignment after max_iter centre updates;
+        # ours are the assignment of round `iters`: the same after one more assignment step
+        C = km.cluster_centers_
+        labels = np.argmin(((X[:, None, :] - C[None]) ** 2).sum(-1), axis=1)
+        _, a_next = O.cluster_keys(Q, K, L, iters + 1)
+        assert np.array_equal(a_next, labels), iters
+
+
+def test_cluster_keys_invariant_to_query_scale_and_blocks_keep_sizes():
+    L, Q, K = _cluster_case()
+    kp, a = O.cluster_keys(Q, K, L, 2)
+    kp2, a2 = O.cluster_keys(Q * 4.0, K, L, 2)
+    assert np.array_equal(a, a2) and np.array_equal(kp, kp2)
+    Nv = int(L.counts[:L.nb_video].sum())
+    assert sorted(kp[:Nv].tolist()) == list(range(Nv))          # a permutation of the video keys
+    assert np.array_equal(kp[Nv:], L.perm[Nv:])                 # padding and text unchanged
+    KL = O.key_layout(L, kp)
+    assert [len(KL.rows(j)) for j in range(L.nb)] == L.counts.tolist()
+    # keys sorted by cluster: the cluster ids along the key order never decrease
+    assert np.all(np.diff(a[kp[:Nv]]) >= 0)
+
+
+def test_cluster_keys_keeps_block_constant_keys_in_their_blocks():
+    # keys constant within each tile block and far apart across blocks: every key stays in its
+    # own block's cluster, so the key blocks are the tile blocks (members in raster order)
+    L, Q, K = _cluster_case(text=0)
+    rng = np.random.default_rng(3)
+    for j in range(L.nb):
+        K[L.rows(j)] = rng.standard_normal(K.shape[1]) * 10.0
+    kp, a = O.cluster_keys(Q, K, L, 3)
+    for j in range(L.nb):
+        assert set(a[L.rows(j)].tolist()) == {j}
+        assert kp[j * L.B:j * L.B + L.counts[j]].tolist() == sorted(L.rows(j).tolist())
+
+
+def test_keys_scored_alike_by_every_query_share_a_cluster():
+    # queries confined to a 3-dimensional subspace: keys that differ only outside it receive
+    # identical scores, are at distance 0 in the query metric, and must land in one cluster
+    L, Q, K = _cluster_case(text=0)
+    Q[:, 3:] = 0.0
+    rng = np.random.default_rng(9)
+    K[40, :] = K[17, :]
+    K[40, 3:] = rng.standard_normal(K.shape[1] - 3) * 50.0
+    _, a = O.cluster_keys(Q, K, L, 2)
+    assert a[40] == a[17]
