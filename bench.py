@@ -374,8 +374,22 @@ def retrieval_accuracy(w, h0, h1, qkv, dev, ws):
     Hl = h1 - h0
     p = torch.tensor(list(w.p[h0:h1]), dtype=torch.float32, device=dev)
     out = {}
-    for name, mode in (("meanpool", bsa.BSA_SCORE_MEANPOOL), ("park", bsa.BSA_SCORE_PARK)):
-        prob = bsa.problem(Hl, w.d, w.T, w.H, w.W, w.text_tokens, w.block, score_mode=mode)
+    # query-aware key blocks (PARK's key side): two k-means rounds, timed with CUDA events
+    base = bsa.problem(Hl, w.d, w.T, w.H, w.W, w.text_tokens, w.block, score_mode=bsa.BSA_SCORE_PARK)
+    bplan = bsa.bsa_plan(base)
+    table = torch.empty(Hl, bplan.npad, dtype=torch.int32, device=dev)
+    cws = torch.empty(bplan.cluster_workspace_bytes, dtype=torch.uint8, device=dev)
+    bsa.bsa_cluster_keys(base, Q, K, 2, table, None, cws)            # warm-up
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    bsa.bsa_cluster_keys(base, Q, K, 2, table, None, cws)
+    e1.record()
+    torch.cuda.synchronize()
+    cluster_ms = max_over_ranks(e0.elapsed_time(e1), ws, dev)
+    del cws
+    for name, mode, ktab in (("meanpool", bsa.BSA_SCORE_MEANPOOL, None), ("park", bsa.BSA_SCORE_PARK, None),
+                             ("park_query_aware_key_blocks", bsa.BSA_SCORE_PARK, table)):
+        prob = bsa.problem(Hl, w.d, w.T, w.H, w.W, w.text_tokens, w.block, score_mode=mode, key_table=ktab)
         plan = bsa.bsa_plan(prob)
         nb = plan.nb
         S = torch.empty(Hl, nb, nb, dtype=torch.float32, device=dev)
@@ -399,8 +413,11 @@ def retrieval_accuracy(w, h0, h1, qkv, dev, ws):
         out[name] = {"captured_mass_mean": round(tot / n, 5), "kept_blocks_per_video_row": round(kept / n, 3)}
         if mn is not None:
             out[name]["captured_mass_min_block"] = round(mn, 5)
+    out["park_query_aware_key_blocks"]["cluster_ms"] = round(cluster_ms, 3)
+    out["park_query_aware_key_blocks"]["cluster_rounds"] = 2
     out["definition"] = ("mean over video query blocks of the share of each query's exact softmax mass held by "
-                         "its top-p kept blocks (bsa_captured_mass)")
+                         "its top-p kept blocks (bsa_captured_mass); park_query_aware_key_blocks: PARK scores "
+                         "over the key blocks of bsa_cluster_keys")
     return out
 
 

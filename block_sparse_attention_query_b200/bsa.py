@@ -34,6 +34,7 @@ class Problem(ctypes.Structure):
         ("text_tokens", ctypes.c_int), ("block", ctypes.c_int),
         ("tile_t", ctypes.c_int), ("tile_h", ctypes.c_int), ("tile_w", ctypes.c_int),
         ("score_mode", ctypes.c_int),
+        ("key_table", ctypes.c_void_p),
     ]
 
 
@@ -47,6 +48,7 @@ class PlanInfo(ctypes.Structure):
         ("drift_workspace_bytes", ctypes.c_size_t),
         ("attention_workspace_bytes", ctypes.c_size_t),
         ("mass_workspace_bytes", ctypes.c_size_t),
+        ("cluster_workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -71,6 +73,9 @@ EXPORTS = {
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                             ctypes.c_void_p]),
+    "bsa_cluster_keys": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
     "bsa_dense_correction": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -111,9 +116,11 @@ def check(status: int, where: str) -> None:
 
 
 def problem(heads, d, T, H, W, text_tokens=0, block=128, tile=(0, 0, 0),
-            score_mode=BSA_SCORE_MEANPOOL) -> Problem:
+            score_mode=BSA_SCORE_MEANPOOL, key_table=None) -> Problem:
+    """key_table: a device int32 tensor [heads, nb*block] from bsa_cluster_keys, or None."""
     return Problem(heads, T * H * W + text_tokens, d, T, H, W, text_tokens, block,
-                   tile[0], tile[1], tile[2], score_mode)
+                   tile[0], tile[1], tile[2], score_mode,
+                   None if key_table is None else key_table.data_ptr())
 
 
 def bsa_plan(prob: Problem) -> PlanInfo:
@@ -173,6 +180,13 @@ def bsa_sparse_attention(prob, Q, K, V, idx, cnt, O, ws, stream=None):
                                    _ptr(O), _ptr(ws),
                                    ws.numel() * ws.element_size() if ws is not None else 0,
                                    _stream(stream)), "bsa_sparse_attention")
+
+
+def bsa_cluster_keys(prob, Q, K, iters, key_table, assignment, ws, stream=None):
+    check(lib.bsa_cluster_keys(ctypes.byref(prob), _ptr(Q), _ptr(K), int(iters), _ptr(key_table), _ptr(assignment),
+                               _ptr(ws),
+                               ws.numel() * ws.element_size() if ws is not None else 0,
+                               _stream(stream)), "bsa_cluster_keys")
 
 
 def bsa_dense_correction(prob, Q, K, V, refresh, O, R, ws, stream=None):

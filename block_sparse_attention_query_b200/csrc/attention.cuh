@@ -94,6 +94,8 @@ struct Params {
     const int* cnt;
     const int* head_mask;   // nullable: heads with head_mask[h] == 0 are skipped, nothing written
     const int* perm;    // [nb*B] raster token of every block slot, -1 = padding
+    const int* kperm;   // nullable, [heads][nb*B]: key-side slot table (query-aware key blocks);
+                        // NULL: keys and values use perm like the queries
     bsa_bf16* O;
     float* lse;         // nullable, [heads][N]: log2 of the row's softmax denominator in log2
                         // units of the scaled logits (-inf when nothing is kept)
@@ -231,20 +233,20 @@ struct RowToks {
 // Tokens of rows [block*B + (lt/CH)*TPT, +TPT); rows beyond the block, and padding slots,
 // read token row 0 of the head: finite values that the softmax masks (keys) or the epilogue
 // never stores (queries).
+// Entries outside [0, N) (padding, or a bad caller-supplied key table) read a row in range.
 template <int D, int ROWS>
-__device__ inline RowToks<D, ROWS> load_tokens(const Params& P, int block, int lt) {
+__device__ inline RowToks<D, ROWS> load_tokens(const int* table, int B, int N, int block, int lt) {
     using RT = RowToks<D, ROWS>;
     RT rt;
     const int r0 = (lt / RT::CH) * RT::TPT;
-    const int B = P.g.B;
 #pragma unroll
     for (int v = 0; v < RT::TPT / 4; ++v) {
         int4 q = make_int4(0, 0, 0, 0);
-        if (r0 + 4 * v < B) q = __ldg(reinterpret_cast<const int4*>(P.perm + block * B + r0 + 4 * v));
-        rt.t[4 * v + 0] = max(q.x, 0);
-        rt.t[4 * v + 1] = max(q.y, 0);
-        rt.t[4 * v + 2] = max(q.z, 0);
-        rt.t[4 * v + 3] = max(q.w, 0);
+        if (r0 + 4 * v < B) q = __ldg(reinterpret_cast<const int4*>(table + block * B + r0 + 4 * v));
+        rt.t[4 * v + 0] = min(max(q.x, 0), N - 1);
+        rt.t[4 * v + 1] = min(max(q.y, 0), N - 1);
+        rt.t[4 * v + 2] = min(max(q.z, 0), N - 1);
+        rt.t[4 * v + 3] = min(max(q.w, 0), N - 1);
     }
     return rt;
 }
@@ -364,8 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
             const int qb = k & 1;
             // tokens of the query block and of the first kept block, and the index of the
             // second kept block, are all in flight before the first wait
-            const RowToks<D, BQ> tq = load_tokens<D, BQ>(P, it.i, lt);
-            RowToks<D, BK> tk = load_tokens<D, BK>(P, kept_block(it, 0), lt);
+            // key and value rows come from the key-side table of this head
+            const int* ktab = P.kperm != nullptr ? P.kperm + (size_t)it.h * nb * g.B : P.perm;
+            const RowToks<D, BQ> tq = load_tokens<D, BQ>(P.perm, g.B, g.N, it.i, lt);
+            RowToks<D, BK> tk = load_tokens<D, BK>(ktab, g.B, g.N, kept_block(it, 0), lt);
             int kb_ahead = it.n > 1 ? kept_block(it, 1) : 0;
             if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch);
             if (!ok) break;
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attention_kernel(Params P)
                 const int ks = gblk % NK, vs = gblk % NV;
                 const RowToks<D, BK> cur = tk;
                 if (j + 1 < it.n) {          // prefetch: next block's tokens, index two ahead
-                    tk = load_tokens<D, BK>(P, kb_ahead, lt);
+                    tk = load_tokens<D, BK>(ktab, g.B, g.N, kb_ahead, lt);
                     if (j + 2 < it.n) kb_ahead = kept_block(it, j + 2);
                 }
                 if (gblk >= NK) ok = mbar_wait(&k_empty[ks], ((gblk / NK) - 1) & 1, epoch);

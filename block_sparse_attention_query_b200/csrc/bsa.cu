@@ -16,6 +16,7 @@
 #include "attention.cuh"
 #include "mass.cuh"
 #include "correct.cuh"
+#include "cluster.cuh"
 
 using namespace bsa;
 
@@ -197,6 +198,16 @@ size_t mass_ws_bytes(const Geom& g) {
     return attention_ws_bytes(g) + align256(rows * g.d * 2) + 2 * align256(rows * sizeof(float));
 }
 
+// Clustering workspace: [M partials: heads*chunks*d*d f32][M: heads*d*d f32][pooled means:
+// 2*heads*nb*d f32][block-slot table][centroids, M c: 2*heads*C*d f32][c.Mc: heads*C f32]
+// [assignment, order: 2*heads*Nv i32][cluster starts: heads*(C+1) i32]
+int qtq_chunks(const Geom& g) { return (g.N + clu::kQtqRows - 1) / clu::kQtqRows; }
+size_t cluster_ws_bytes(const Geom& g) {
+    const size_t h = g.heads, d = g.d, C = g.nbv, Nv = g.Nv;
+    return align256(h * qtq_chunks(g) * d * d * 4) + align256(h * d * d * 4) + pooled_bytes(g) + perm_bytes(g) +
+           2 * align256(h * C * d * 4) + align256(h * C * 4) + 2 * align256(h * Nv * 4) + align256(h * (C + 1) * 4);
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -231,9 +242,11 @@ int launch_attention(const attn::Params& P, cudaStream_t st) {
 }
 
 attn::Params attention_params(const Geom& g, const bsa_bf16* Q, const bsa_bf16* K, const bsa_bf16* V,
-                              const int* idx, const int* cnt, bsa_bf16* O, float* lse, void* ws) {
+                              const int* idx, const int* cnt, bsa_bf16* O, float* lse, void* ws,
+                              const int* key_table) {
     attn::Params P;
     P.g = g;
+    P.kperm = key_table;
     P.Q = Q;
     P.K = K;
     P.V = V;
@@ -253,6 +266,40 @@ attn::Params attention_params(const Geom& g, const bsa_bf16* Q, const bsa_bf16* 
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
     P.n_items = P.n_text_items + g.heads * g.nbv;
     return P;
+}
+
+template <int D>
+int run_cluster(const Geom& g, const bsa_bf16* Q, const bsa_bf16* K, int iters, int nchunks, float* part,
+                float* M, const float* kbar, float* cent, float* Wc, float* bvec, int* assign, int* order,
+                int* start, int* key_table, cudaStream_t st) {
+    int rc;
+    const int C = g.nbv, Nv = g.Nv;
+    clu::qtq_partial_kernel<D><<<dim3(nchunks, g.heads), clu::kQtqThreads, 0, st>>>(Q, g.N, part);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    clu::qtq_reduce_kernel<D><<<g.heads, 256, 0, st>>>(part, nchunks, g.N, M);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    clu::centroid_init_kernel<D><<<dim3(C, g.heads), D, 0, st>>>(kbar, g.nb, C, cent);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    constexpr int KS = D + 4;
+    const int asmem = (clu::kAssignKeys * KS + clu::kAssignChunk * KS + clu::kAssignChunk +
+                       2 * 8 * clu::kAssignKeys) * 4;
+    if (cudaFuncSetAttribute(clu::assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, asmem) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    const dim3 agrid((Nv + clu::kAssignKeys - 1) / clu::kAssignKeys, g.heads);
+    for (int t = 0; t < iters; ++t) {
+        clu::centroid_prep_kernel<D><<<dim3(C, g.heads), D, 0, st>>>(M, cent, C, Wc, bvec);
+        if ((rc = launch_status()) != BSA_OK) return rc;
+        clu::assign_kernel<D><<<agrid, clu::kAssignThreads, asmem, st>>>(K, g.N, Nv, Wc, bvec, C, assign);
+        if ((rc = launch_status()) != BSA_OK) return rc;
+        clu::cluster_sort_kernel<<<g.heads, 32, 2 * (C + 1) * sizeof(int), st>>>(assign, Nv, C, order, start);
+        if ((rc = launch_status()) != BSA_OK) return rc;
+        if (t + 1 < iters) {
+            clu::centroid_update_kernel<D><<<dim3(C, g.heads), D, 0, st>>>(K, g.N, Nv, C, order, start, cent);
+            if ((rc = launch_status()) != BSA_OK) return rc;
+        }
+    }
+    clu::key_table_kernel<<<dim3((g.nb * g.B + 255) / 256, g.heads), 256, 0, st>>>(g, order, key_table);
+    return launch_status();
 }
 
 int run_attention(const attn::Params& P, cudaStream_t st) {
@@ -285,6 +332,7 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
     info.attention_workspace_bytes = attention_ws_bytes(g);
     info.mass_workspace_bytes = mass_ws_bytes(g);
+    info.cluster_workspace_bytes = cluster_ws_bytes(g);
     *out = info;
     return BSA_OK;
 }
@@ -305,7 +353,9 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     int rc = make_geom(prob, &g);
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || scores == nullptr) return BSA_ERR_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(head_mask)) return BSA_ERR_ALIGN;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(head_mask) ||
+        !aligned16(prob->key_table))
+        return BSA_ERR_ALIGN;
     if (ws == nullptr || ws_bytes < score_ws_bytes(g, prob->score_mode)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -316,10 +366,11 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(g, perm);
     if ((rc = launch_status()) != BSA_OK) return rc;
     const dim3 pgrid(g.nb, g.heads);
-    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
-    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
-    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
-    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, head_mask, qbar, kbar);
+    const int* kperm = prob->key_table;
+    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
+    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
+    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
+    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
     if ((rc = launch_status()) != BSA_OK) return rc;
     bsa_bf16* ksplit = reinterpret_cast<bsa_bf16*>(static_cast<uint8_t*>(ws) + pooled_bytes(g) + perm_bytes(g));
     if (prob->score_mode == BSA_SCORE_MEANPOOL && (long long)g.heads * mp_nbq(g) / mp::BQ < sm_count()) {
@@ -428,13 +479,54 @@ int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr) return BSA_ERR_ARG;
     if ((idx == nullptr) != (cnt == nullptr)) return BSA_ERR_ARG;   // both NULL: dense
+    if (!aligned16(prob->key_table)) return BSA_ERR_ALIGN;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(cnt) || !aligned16(O))
         return BSA_ERR_ALIGN;
     const size_t need = attention_ws_bytes(g);
     if (ws == nullptr || ws_bytes < need) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
-    const attn::Params P = attention_params(g, Q, K, V, idx, cnt, O, nullptr, ws);
+    const attn::Params P = attention_params(g, Q, K, V, idx, cnt, O, nullptr, ws, prob->key_table);
     return run_attention(P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_cluster_keys(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K, int iters,
+                     int* key_table, int* assignment, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+    Geom g;
+    int rc = make_geom(prob, &g);
+    if (rc != BSA_OK) return rc;
+    if (Q == nullptr || K == nullptr || key_table == nullptr) return BSA_ERR_ARG;
+    if (iters < 1 || iters > 64 || g.nbv < 1) return BSA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(key_table) || !aligned16(assignment)) return BSA_ERR_ALIGN;
+    if (ws == nullptr || ws_bytes < cluster_ws_bytes(g)) return BSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BSA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t h = g.heads, d = g.d, C = g.nbv, Nv = g.Nv;
+    const int nchunks = qtq_chunks(g);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    float* part = reinterpret_cast<float*>(w);                        w += align256(h * nchunks * d * d * 4);
+    float* M = reinterpret_cast<float*>(w);                           w += align256(h * d * d * 4);
+    float* qbar = reinterpret_cast<float*>(w);
+    float* kbar = qbar + h * g.nb * d;                                w += pooled_bytes(g);
+    int* perm = reinterpret_cast<int*>(w);                            w += perm_bytes(g);
+    float* cent = reinterpret_cast<float*>(w);                        w += align256(h * C * d * 4);
+    float* Wc = reinterpret_cast<float*>(w);                          w += align256(h * C * d * 4);
+    float* bvec = reinterpret_cast<float*>(w);                        w += align256(h * C * 4);
+    int* assign = assignment != nullptr ? assignment : reinterpret_cast<int*>(w);
+    w += align256(h * Nv * 4);
+    int* order = reinterpret_cast<int*>(w);                           w += align256(h * Nv * 4);
+    int* start = reinterpret_cast<int*>(w);
+    perm_kernel<<<(g.nb * g.B + 255) / 256, 256, 0, st>>>(g, perm);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    const dim3 pgrid(g.nb, g.heads);
+    if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, nullptr, nullptr, qbar, kbar);
+    else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, nullptr, nullptr, qbar, kbar);
+    else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, nullptr, nullptr, qbar, kbar);
+    else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, nullptr, nullptr, qbar, kbar);
+    if ((rc = launch_status()) != BSA_OK) return rc;
+    return g.d == 128 ? run_cluster<128>(g, Q, K, iters, nchunks, part, M, kbar, cent, Wc, bvec, assign, order,
+                                         start, key_table, st)
+                      : run_cluster<64>(g, Q, K, iters, nchunks, part, M, kbar, cent, Wc, bvec, assign, order,
+                                        start, key_table, st);
 }
 
 int bsa_dense_correction(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
@@ -445,13 +537,14 @@ int bsa_dense_correction(const bsa_problem* prob, const bsa_bf16* Q, const bsa_b
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || V == nullptr || refresh == nullptr || O == nullptr || R == nullptr)
         return BSA_ERR_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(refresh) || !aligned16(O) || !aligned16(R))
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(refresh) || !aligned16(O) || !aligned16(R) ||
+        !aligned16(prob->key_table))
         return BSA_ERR_ALIGN;
     if (ws == nullptr || ws_bytes < attention_ws_bytes(g)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // dense attention of the refreshed heads, written into their rows of R
-    attn::Params P = attention_params(g, Q, K, V, nullptr, nullptr, R, nullptr, ws);
+    attn::Params P = attention_params(g, Q, K, V, nullptr, nullptr, R, nullptr, ws, prob->key_table);
     P.head_mask = refresh;
     if ((rc = run_attention(P, st)) != BSA_OK) return rc;
     const long long elems = (long long)g.N * g.d;
@@ -466,7 +559,8 @@ int bsa_captured_mass(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16
     int rc = make_geom(prob, &g);
     if (rc != BSA_OK) return rc;
     if (Q == nullptr || K == nullptr || idx == nullptr || cnt == nullptr || mass == nullptr) return BSA_ERR_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(idx) || !aligned16(cnt) || !aligned16(mass))
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(idx) || !aligned16(cnt) || !aligned16(mass) ||
+        !aligned16(prob->key_table))
         return BSA_ERR_ALIGN;
     if (ws == nullptr || ws_bytes < mass_ws_bytes(g)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
@@ -478,9 +572,9 @@ int bsa_captured_mass(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16
     float* lse_all = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lse_kept) + align256(rows * sizeof(float)));
     // the log-sum-exp over the kept keys, then over every key; the outputs themselves are not
     // needed, so K stands in for V
-    attn::Params P = attention_params(g, Q, K, K, idx, cnt, o_scratch, lse_kept, ws);
+    attn::Params P = attention_params(g, Q, K, K, idx, cnt, o_scratch, lse_kept, ws, prob->key_table);
     if ((rc = run_attention(P, st)) != BSA_OK) return rc;
-    P = attention_params(g, Q, K, K, nullptr, nullptr, o_scratch, lse_all, ws);
+    P = attention_params(g, Q, K, K, nullptr, nullptr, o_scratch, lse_all, ws, prob->key_table);
     if ((rc = run_attention(P, st)) != BSA_OK) return rc;
     mass_kernel<<<dim3(g.nb, g.heads), kMassThreads, 0, st>>>(g, P.perm, lse_kept, lse_all, mass);
     return launch_status();

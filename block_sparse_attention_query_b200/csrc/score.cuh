@@ -27,10 +27,13 @@ __device__ inline void accum_bf16x8(float (&acc)[8], const uint4& v) {
 }
 
 // grid (nb, heads), 256 threads. Pools Q and K of block i, head h into qbar/kbar [heads][nb][D].
+// kperm (nullable): per-head key-side block-slot table [heads][nb*B] (query-aware key
+// blocks); NULL: keys use the tile layout like the queries.
 template <int D, int B>
 __global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __restrict__ Q,
                                                    const bsa_bf16* __restrict__ K,
                                                    const int* __restrict__ perm,
+                                                   const int* __restrict__ kperm,
                                                    const int* __restrict__ head_mask,
                                                    float* __restrict__ qbar, float* __restrict__ kbar) {
     constexpr int CH = D / 8;               // 16-byte chunks per row
@@ -41,20 +44,20 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const bsa_bf16* __res
     const int c = threadIdx.x % CH, rs = threadIdx.x / CH;
     const size_t head_off = (size_t)h * g.N * D;
 
-    int tok[NIT];
+    int tok[NIT], tokk[NIT];
+    const int* kp = kperm != nullptr ? kperm + (size_t)h * g.nb * B : perm;
 #pragma unroll
-    for (int k = 0; k < NIT; ++k) tok[k] = __ldg(perm + i * B + rs + k * RPP);
+    for (int k = 0; k < NIT; ++k) {
+        tok[k] = __ldg(perm + i * B + rs + k * RPP);
+        tokk[k] = min(__ldg(kp + i * B + rs + k * RPP), g.N - 1);   // a bad caller table stays in range
+    }
     uint4 vq[NIT], vk[NIT];
 #pragma unroll
     for (int k = 0; k < NIT; ++k) {
-        if (tok[k] >= 0) {
-            const size_t off = head_off + (size_t)tok[k] * D + c * 8;
-            vq[k] = __ldg(reinterpret_cast<const uint4*>(Q + off));
-            vk[k] = __ldg(reinterpret_cast<const uint4*>(K + off));
-        } else {
-            vq[k] = make_uint4(0, 0, 0, 0);
-            vk[k] = make_uint4(0, 0, 0, 0);
-        }
+        vq[k] = tok[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(Q + head_off + (size_t)tok[k] * D + c * 8))
+                            : make_uint4(0, 0, 0, 0);
+        vk[k] = tokk[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(K + head_off + (size_t)tokk[k] * D + c * 8))
+                             : make_uint4(0, 0, 0, 0);
     }
     float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll

@@ -81,6 +81,13 @@ typedef struct bsa_problem {
     int tile_t, tile_h, tile_w;  /* tile shape; all 0 = default (1x8x8 for 64, 2x8x8 for 128);
                                     otherwise tile_t*tile_h*tile_w must equal block */
     int score_mode;     /* BSA_SCORE_MEANPOOL or BSA_SCORE_PARK */
+    const int* key_table;   /* DEVICE pointer, nullable: per-head key-side block-slot table
+                               [heads][nb*block] written by bsa_cluster_keys (query-aware key
+                               blocks). When set, bsa_score_blocks pools keys and
+                               bsa_sparse_attention / bsa_captured_mass gather keys and values
+                               through it; queries always use the tile layout. NULL: keys use
+                               the tile layout too. Entries outside [-1, tokens) are clamped
+                               into range (a wrong table gives wrong results, never a fault). */
 } bsa_problem;
 
 /* Derived sizes, filled by bsa_plan (host only, no CUDA call). */
@@ -94,6 +101,7 @@ typedef struct bsa_plan_info {
     size_t drift_workspace_bytes;      /* bsa_drift_check */
     size_t attention_workspace_bytes;  /* bsa_sparse_attention */
     size_t mass_workspace_bytes;       /* bsa_captured_mass */
+    size_t cluster_workspace_bytes;    /* bsa_cluster_keys */
 } bsa_plan_info;
 
 /* Validate `prob` and fill `out`. Host only; launches nothing.
@@ -191,6 +199,28 @@ int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bs
 int bsa_sparse_attention(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                          const bsa_bf16* V, const int* idx, const int* cnt, bsa_bf16* O,
                          void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Query-aware key blocks (PARK, Abstract: keys are transformed with information from the
+ * current queries before clustering, so that keys receiving similar QK scores are grouped
+ * together). Per head: M = Q^T Q / tokens over the real queries, so (k1-k2)^T M (k1-k2) is the
+ * mean-square difference of the scores the queries give two keys; Lloyd's k-means with that
+ * metric over the video keys, one cluster per video block, started from the tile-block means;
+ * each of `iters` rounds assigns every key to argmin_j (k-c_j)^T M (k-c_j) (ties to the lowest
+ * j) and, except in the last round, moves each non-empty cluster's centroid to the mean of
+ * its keys. The table lists the video keys in (cluster, raster index) order followed by the
+ * tile layout's padding and text slots: cut every `block` keys it gives key blocks of the same
+ * sizes as the tile layout. Pass it as prob->key_table to the scoring and attention calls.
+ *   Q, K        [heads, tokens, d] bf16, raster order.
+ *   iters       1..64 rounds.
+ *   key_table   [heads, nb*block] int32 out (raster token per slot, -1 = padding).
+ *   assignment  [heads, T*H*W] int32 out, nullable: cluster of every video key (raster order)
+ *               in the last round.
+ *   ws          at least plan.cluster_workspace_bytes (M and its partial sums, centroids, the
+ *               assignment and the sorted order). prob->key_table is ignored here.
+ * Deterministic (fixed summation orders). Not a per-step call: it costs a pass over Q (M) and
+ * heads x video keys x clusters x d multiply-adds per round. */
+int bsa_cluster_keys(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K, int iters,
+                     int* key_table, int* assignment, void* ws, size_t ws_bytes, bsa_stream_t stream);
 
 /* Cached dense correction of this step's sparse output (RECAP: Reciprocal Sparse Attention
  * and Hierarchical Caching for Efficient Video Diffusion, Abstract: a cached dense refinement

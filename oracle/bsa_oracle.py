@@ -518,7 +518,7 @@ def query_metric(Qh: np.ndarray, layout: Layout) -> np.ndarray:
     return Q.T @ Q / len(rows)
 
 
-def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2):
+def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2, with_objective: bool = False):
     """Query-aware key blocks (PARK abstract, key-side clustering).
 
     Readings (the page gives no formula): the video keys are clustered by Lloyd's k-means
@@ -528,7 +528,9 @@ def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2)
     every non-empty cluster's centroid to the mean of its keys. The key blocks then follow the
     block rule of the query side: the video keys in order of (cluster, raster index), cut every
     B keys (so every key block keeps its tile-layout size); text key blocks are unchanged.
-    Returns (key_perm int64 [nb*B] like Layout.perm, assignment int64 [Nv] of the last round).
+    Returns (key_perm int64 [nb*B] like Layout.perm, assignment int64 [Nv] of the last round)
+    and, with `with_objective`, the last round's objective [Nv, nb_video] and the magnitude of
+    its terms (|b_j| + 2 sum_c |k_c w_jc|, for error bounds).
     """
     if iters < 1:
         raise ValueError("iters >= 1")
@@ -537,7 +539,7 @@ def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2)
     Nv = int(layout.counts[:nv].sum())
     Kv = Kh[:Nv]
     C = np.stack([Kh[layout.rows(j)].mean(axis=0) for j in range(nv)])
-    a = None
+    a = obj = W = b = None
     for _ in range(iters):
         W = C @ M                                   # w_j = M c_j  (M symmetric)
         b = (C * W).sum(axis=1)                     # c_j^T M c_j
@@ -550,6 +552,9 @@ def cluster_keys(Qh: np.ndarray, Kh: np.ndarray, layout: Layout, iters: int = 2)
     order = np.lexsort((np.arange(Nv), a))          # by cluster, then raster index
     key_perm = layout.perm.copy()
     key_perm[:Nv] = order
+    if with_objective:
+        scale = np.abs(b)[None, :] + 2.0 * (np.abs(Kv) @ np.abs(W).T)
+        return key_perm, a, obj, scale
     return key_perm, a
 
 

@@ -71,13 +71,16 @@ def bf16_bits_f64(bits):
 
 # ------------------------------------------------------------------ score error bound
 
-def score_bound(Qh: np.ndarray, Kh: np.ndarray, layout, mode: str, S: np.ndarray | None = None) -> np.ndarray:
+def score_bound(Qh: np.ndarray, Kh: np.ndarray, layout, mode: str, S: np.ndarray | None = None,
+                klayout=None) -> np.ndarray:
     """Absolute error bound [nb, nb] of a float32 kernel's block scores for one head
-    (float64 Q, K [N, d] in raster order); S are the exact scores if already computed."""
+    (float64 Q, K [N, d] in raster order); S are the exact scores if already computed;
+    klayout: the key-side layout when keys are blocked differently (query-aware key blocks)."""
     d = Qh.shape[1]
     s = 1.0 / math.sqrt(d)
-    kbar = O.pool_blocks(Kh, layout)
-    kabs = O.pool_blocks(np.abs(Kh), layout)
+    kl = layout if klayout is None else klayout
+    kbar = O.pool_blocks(Kh, kl)
+    kabs = O.pool_blocks(np.abs(Kh), kl)
     nb = layout.nb
     if mode == "meanpool":
         qbar = O.pool_blocks(Qh, layout)
@@ -85,7 +88,9 @@ def score_bound(Qh: np.ndarray, Kh: np.ndarray, layout, mode: str, S: np.ndarray
         E = s * (K_DOT * (np.abs(qbar) @ np.abs(kbar).T)
                  + K_POOL * (qabs @ np.abs(kbar).T + np.abs(qbar) @ kabs.T))
         if S is None:
-            S = O.score_meanpool(Qh, Kh, layout)
+            S = O.score_meanpool(Qh, Kh, layout) if klayout is None else None
+        if S is None:
+            raise ValueError("pass the exact scores for a separate key layout")
         return S * U32 * (E + (S * E).sum(axis=1, keepdims=True) + k_norm(nb))
     if mode == "park":
         out = np.zeros((nb, nb))

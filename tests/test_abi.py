@@ -120,4 +120,20 @@ def test_calls_reject_bad_pointers_before_launch():
     assert L.bsa_dense_correction(pr, a, a, a, None, a, a, a, aw, None) == bsa.BSA_ERR_ARG
     assert L.bsa_dense_correction(pr, a, a, a, a, a, mis, a, aw, None) == bsa.BSA_ERR_ALIGN
     assert L.bsa_dense_correction(pr, a, a, a, a, a, a, a, aw - 1, None) == bsa.BSA_ERR_WORKSPACE
+    # query-aware key blocks: iteration range, pointers, alignment, workspace; a misaligned key
+    # table in the problem is refused by the calls that read it
+    cw = bsa.bsa_plan(prob).cluster_workspace_bytes
+    assert cw > 0
+    assert L.bsa_cluster_keys(pr, a, a, 0, a, None, a, cw, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_cluster_keys(pr, a, a, 65, a, None, a, cw, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_cluster_keys(pr, a, a, 2, None, None, a, cw, None) == bsa.BSA_ERR_ARG
+    assert L.bsa_cluster_keys(pr, a, a, 2, mis, None, a, cw, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_cluster_keys(pr, a, a, 2, a, mis, a, cw, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_cluster_keys(pr, a, a, 2, a, None, a, cw - 1, None) == bsa.BSA_ERR_WORKSPACE
+    bad = bsa.problem(2, 64, 4, 16, 16, 0, 64)
+    bad.key_table = 4096 + 4
+    pb = ctypes.byref(bad)
+    assert L.bsa_score_blocks(pb, a, a, None, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_sparse_attention(pb, a, a, a, a, a, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_captured_mass(pb, a, a, a, a, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
     assert bsa.bsa_launch_count() == launches_before     # none of the rejected calls launched

@@ -605,3 +605,105 @@ def test_dense_correction_heads_masked():
     mx, rel = PT.attention_errors(out[1], dense, np.arange(c.N))
     assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2
     assert np.abs(Rn[1] - (out[1] - sparse[1])).max() <= 2 ** -8 * np.abs(out[1] - sparse[1]).max() + 1e-6
+
+
+# ------------------------------------------------------------ query-aware key blocks
+# The GPU's k-means rounds run in float32; a key may be assigned differently from the float64
+# oracle only where the oracle's objective of the GPU's choice lies within 1e-4 of the terms'
+# magnitude (|b_j| + 2 sum |k w_j|) of its own optimum: a float32 near-tie (such a flip can move
+# a few other keys in later rounds, so at most 0.5% of the keys may differ).
+CLUSTER_REL = 1e-4
+
+
+def _gpu_cluster(c, iters):
+    bsa = _bsa()
+    table = torch.full((c.heads, c.nb * c.B), -9, dtype=torch.int32, device="cuda")
+    nv = c.layout.nb_video
+    Nv = int(c.layout.counts[:nv].sum())
+    assign = torch.full((c.heads, Nv), -9, dtype=torch.int32, device="cuda")
+    bsa.bsa_cluster_keys(c.prob, c.Q, c.K, iters, table, assign, c.ws(c.plan.cluster_workspace_bytes))
+    _status_ok()
+    return table, assign
+
+
+def _check_clustering(c, h, table_h, assign_h, iters):
+    L = c.layout
+    kp, a, obj, scale = O.cluster_keys(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]), L, iters, with_objective=True)
+    Nv = len(a)
+    # the table is the GPU's own assignment sorted by (cluster, raster index), then the tile
+    # layout's padding and text slots: exactly
+    assert np.array_equal(table_h[:Nv], np.lexsort((np.arange(Nv), assign_h)))
+    assert np.array_equal(table_h[Nv:], L.perm[Nv:])
+    diff = np.nonzero(assign_h != a)[0]
+    u = np.arange(Nv)
+    gap = obj[u, assign_h] - obj[u, a]
+    near = gap <= CLUSTER_REL * scale[u, assign_h]
+    assert np.all(near[diff]), (h, diff[~near[diff]][:5], gap[diff][:5])
+    assert len(diff) <= max(2, Nv // 200), (h, len(diff))
+    return len(diff), kp
+
+
+@pytest.mark.parametrize("name", ["tiny", "text_d128_b128", "ragged_d128_b64"])
+@pytest.mark.parametrize("iters", [1, 3])
+def test_cluster_keys_matches_oracle(name, iters):
+    c = Case(**SMALL[name])
+    table, assign = _gpu_cluster(c, iters)
+    table, assign = table.cpu().numpy(), assign.cpu().numpy()
+    flips = [_check_clustering(c, h, table[h], assign[h], iters)[0] for h in range(c.heads)]
+    print(f"\n[key clustering] {name}, {iters} rounds: assignments differing from the oracle {flips}")
+
+
+@pytest.mark.parametrize("mode", ["park", "meanpool"])
+def test_scores_and_attention_through_key_table(mode):
+    # scores, masks and attention with the GPU's query-aware key blocks against the oracle on
+    # the same key table
+    bsa = _bsa()
+    c = Case(**SMALL["text_d128_b128"], mode=mode)
+    table, _ = _gpu_cluster(c, 2)
+    smode = bsa.BSA_SCORE_PARK if mode == "park" else bsa.BSA_SCORE_MEANPOOL
+    c.prob = bsa.problem(c.heads, c.d, 6, 20, 24, 256, c.B, score_mode=smode, key_table=table)
+    S = c.gpu_scores()
+    idx, cnt = c.gpu_select(S)
+    _status_ok()
+    S, idx_h, cnt_h, tab = S.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), table.cpu().numpy()
+    S_or = np.zeros_like(S)
+    bounds = []
+    oracle_masks = []
+    for h in range(c.heads):
+        Qh, Kh = O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h])
+        KL = O.key_layout(c.layout, tab[h])
+        if mode == "park":
+            ref = O.score_park_keys(Qh, Kh, c.layout, KL)
+        else:
+            ref = O._softmax_rows(O.pool_blocks(Qh, c.layout) @ O.pool_blocks(Kh, KL).T / math.sqrt(c.d))
+        bnd = PT.score_bound(Qh, Kh, c.layout, mode, ref if mode == "meanpool" else None, klayout=KL)
+        _check_scores(S[h], ref, bnd, ("key table", mode, h))
+        S_or[h] = ref.astype(np.float32)
+        bounds.append(bnd)
+        oracle_masks.append(O.select_topp(S_or[h], c.p[h], c.layout))
+    res = PT.compare_masks(idx_h, cnt_h, S_or, c.p, c.layout, bounds=bounds)
+    _report(f"key table, {mode}", res)
+    assert res["mismatch"] == 0 and res["exempt"] <= PT.exempt_limit(res["rows"]), res
+    # attention on the oracle's mask, keys and values gathered through the table
+    io = np.stack([m[0] for m in oracle_masks]); co = np.stack([m[1] for m in oracle_masks])
+    Od = c.gpu_attention(torch.from_numpy(io).cuda(), torch.from_numpy(co).cuda())
+    _status_ok()
+    got = PT.bf16_bits_f64(PT.from_dev_bf16(Od))
+    for h in range(c.heads):
+        KL = O.key_layout(c.layout, tab[h])
+        ref = O.sparse_attention_keys(O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]), O.bf16_to_f64(c.Vb[h]),
+                                      io[h], co[h], c.layout, KL)
+        mx, rel = PT.attention_errors(got[h], ref, np.arange(c.N))
+        assert mx <= ATT_MAX_ABS and rel <= ATT_REL_L2, (h, mx, rel)
+
+
+@pytest.mark.slow
+def test_full_size_cluster_keys_sampled():
+    # the 480p layer, 2 rounds: assignment near-tie rule on every key of two heads, the table
+    # exact against the GPU's assignment
+    c = _full_case("wan13b_480p", "park")
+    table, assign = _gpu_cluster(c, 2)
+    table, assign = table.cpu().numpy(), assign.cpu().numpy()
+    for h in (0, c.heads - 1):
+        n, _ = _check_clustering(c, h, table[h], assign[h], 2)
+        print(f"\n[key clustering] wan13b_480p head {h}: {n} assignments differ from the oracle")
