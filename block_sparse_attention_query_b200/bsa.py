@@ -35,6 +35,7 @@ class Problem(ctypes.Structure):
         ("tile_t", ctypes.c_int), ("tile_h", ctypes.c_int), ("tile_w", ctypes.c_int),
         ("score_mode", ctypes.c_int),
         ("key_table", ctypes.c_void_p),
+        ("block_means", ctypes.c_void_p),
     ]
 
 
@@ -116,11 +117,13 @@ def check(status: int, where: str) -> None:
 
 
 def problem(heads, d, T, H, W, text_tokens=0, block=128, tile=(0, 0, 0),
-            score_mode=BSA_SCORE_MEANPOOL, key_table=None) -> Problem:
-    """key_table: a device int32 tensor [heads, nb*block] from bsa_cluster_keys, or None."""
+            score_mode=BSA_SCORE_MEANPOOL, key_table=None, block_means=None) -> Problem:
+    """key_table: a device int32 tensor [heads, nb*block] from bsa_cluster_keys, or None.
+    block_means: a device float32 tensor [2, heads, nb, d] (drift pass writes, scores read), or None."""
     return Problem(heads, T * H * W + text_tokens, d, T, H, W, text_tokens, block,
                    tile[0], tile[1], tile[2], score_mode,
-                   None if key_table is None else key_table.data_ptr())
+                   None if key_table is None else key_table.data_ptr(),
+                   None if block_means is None else block_means.data_ptr())
 
 
 def bsa_plan(prob: Problem) -> PlanInfo:

@@ -177,6 +177,14 @@ int drift_chunks(const Geom& g) {
     return (int)((elems + kDriftChunkElems - 1) / kDriftChunkElems);
 }
 
+// Drift workspace: [float64 partial sums: heads * max(chunks, nb) * 4][block-slot table (fused
+// path with bsa_problem.block_means)]
+size_t drift_part_bytes(const Geom& g) {
+    const int parts = drift_chunks(g) > g.nb ? drift_chunks(g) : g.nb;
+    return align256((size_t)g.heads * parts * 4 * sizeof(double));
+}
+size_t drift_ws_bytes(const Geom& g) { return drift_part_bytes(g) + perm_bytes(g); }
+
 int text_splits(const Geom& g) { return (g.nb + attn::kTextChunk - 1) / attn::kTextChunk; }
 
 // Attention workspace: [perm: nb*B int32][text partial O: items*BQ*d fp32][text lse: items*BQ fp32]
@@ -329,7 +337,7 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.tile_h = g.th;
     info.tile_w = g.tw;
     info.score_workspace_bytes = score_ws_bytes(g, prob->score_mode);
-    info.drift_workspace_bytes = (size_t)g.heads * drift_chunks(g) * 4 * sizeof(double);
+    info.drift_workspace_bytes = drift_ws_bytes(g);
     info.attention_workspace_bytes = attention_ws_bytes(g);
     info.mass_workspace_bytes = mass_ws_bytes(g);
     info.cluster_workspace_bytes = cluster_ws_bytes(g);
@@ -359,19 +367,23 @@ int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16*
     if (ws == nullptr || ws_bytes < score_ws_bytes(g, prob->score_mode)) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    float* qbar = static_cast<float*>(ws);
+    if (!aligned16(prob->block_means)) return BSA_ERR_ALIGN;
+    // block means: from the drift pass of this step (bsa_problem.block_means), else pooled here
+    float* qbar = prob->block_means != nullptr ? prob->block_means : static_cast<float*>(ws);
     float* kbar = qbar + (size_t)g.heads * g.nb * g.d;
     int* perm = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pooled_bytes(g));
     const int total = g.nb * g.B;
     perm_kernel<<<(total + 255) / 256, 256, 0, st>>>(g, perm);
     if ((rc = launch_status()) != BSA_OK) return rc;
     const dim3 pgrid(g.nb, g.heads);
+    if (prob->block_means == nullptr) {
     const int* kperm = prob->key_table;
     if (g.d == 128 && g.B == 128) pool_kernel<128, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
     else if (g.d == 128) pool_kernel<128, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
     else if (g.B == 128) pool_kernel<64, 128><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
     else pool_kernel<64, 64><<<pgrid, 256, 0, st>>>(g, Q, K, perm, kperm, head_mask, qbar, kbar);
     if ((rc = launch_status()) != BSA_OK) return rc;
+    }
     bsa_bf16* ksplit = reinterpret_cast<bsa_bf16*>(static_cast<uint8_t*>(ws) + pooled_bytes(g) + perm_bytes(g));
     if (prob->score_mode == BSA_SCORE_MEANPOOL && (long long)g.heads * mp_nbq(g) / mp::BQ < sm_count()) {
         // fewer 128-row items than SMs: the CUDA-core scorer with 8-32 rows per CTA
@@ -453,21 +465,43 @@ int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* 
     if (!aligned16(Q) || !aligned16(K) || !aligned16(Q_ref) || !aligned16(K_ref) || !aligned16(drift) ||
         !aligned16(refresh))
         return BSA_ERR_ALIGN;
+    if (!aligned16(prob->block_means) || !aligned16(prob->key_table)) return BSA_ERR_ALIGN;
     const int chunks = drift_chunks(g);
-    const size_t need = (size_t)g.heads * chunks * 4 * sizeof(double);
+    const bool fused = prob->block_means != nullptr;
+    const size_t need = fused ? drift_ws_bytes(g) : (size_t)g.heads * chunks * 4 * sizeof(double);
     if (ws == nullptr || ws_bytes < need) return BSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return BSA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const long long elems = (long long)g.N * g.d;
-    const dim3 grid(chunks, g.heads);
     double* part = static_cast<double*>(ws);
-    drift_partial_kernel<<<grid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, part);
-    int r2 = launch_status();
-    if (r2 != BSA_OK) return r2;
+    int nparts = chunks;
+    int r2;
+    if (fused) {
+        // one pass over Q, K, Q_ref, K_ref block by block: the drift sums and the block means
+        int* perm = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + drift_part_bytes(g));
+        perm_kernel<<<(g.nb * g.B + 255) / 256, 256, 0, st>>>(g, perm);
+        if ((r2 = launch_status()) != BSA_OK) return r2;
+        float* qbar = prob->block_means;
+        float* kbar = qbar + (size_t)g.heads * g.nb * g.d;
+        const dim3 pgrid(g.nb, g.heads);
+        const int f = force_all ? 1 : 0;
+        const int* kp = prob->key_table;
+#define BSA_DP(DD, BB) drift_pool_kernel<DD, BB><<<pgrid, kDriftPoolThreads, 0, st>>>(g, Q, K, Q_ref, K_ref, perm, kp, f, part, qbar, kbar)
+        if (g.d == 128 && g.B == 128) BSA_DP(128, 128);
+        else if (g.d == 128) BSA_DP(128, 64);
+        else if (g.B == 128) BSA_DP(64, 128);
+        else BSA_DP(64, 64);
+#undef BSA_DP
+        nparts = g.nb;
+    } else {
+        drift_partial_kernel<<<dim3(chunks, g.heads), kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems,
+                                                                             force_all ? 1 : 0, part);
+    }
+    if ((r2 = launch_status()) != BSA_OK) return r2;
     // with force_all the snapshot was taken in the first pass: one CTA per head publishes
     const dim3 fgrid(force_all ? 1 : chunks, g.heads);
     drift_finalize_kernel<<<fgrid, kDriftThreads, 0, st>>>(Q, K, Q_ref, K_ref, elems, force_all ? 1 : 0, tau,
-                                                          part, drift, refresh, chunks);
+                                                          part, drift, refresh, nparts);
     return launch_status();
 }
 
@@ -634,8 +668,11 @@ int bsa_drift_check_noalloc(const bsa_problem* prob, const bsa_bf16* Q, const bs
     const int sc = noalloc_scratch(&scratch);
     if (sc != BSA_OK) return sc;
     // every partial that the finalize pass reads is written first by the partial pass of
-    // the same call, so the shared array needs no clearing between calls
-    return bsa_drift_check(prob, Q, K, Q_ref, K_ref, tau, force_all, drift, refresh, scratch,
+    // the same call, so the shared array needs no clearing between calls; the block means of a
+    // fused pass are not written by this entry point (its scratch holds only the partials)
+    bsa_problem p = *prob;
+    p.block_means = nullptr;
+    return bsa_drift_check(&p, Q, K, Q_ref, K_ref, tau, force_all, drift, refresh, scratch,
                            kNoallocDriftDoubles * sizeof(double), stream);
 }
 

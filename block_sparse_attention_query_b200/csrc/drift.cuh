@@ -5,6 +5,9 @@
 // drift_partial_kernel  grid (chunks, heads): streams Q, K, Q_ref, K_ref once with 16-byte
 //   loads and writes four float64 partial sums per chunk (|Q-Qref|^2, |Qref|^2, |K-Kref|^2,
 //   |Kref|^2). With force_all it also writes the new reference in the same pass.
+// drift_pool_kernel     grid (nb, heads), the same sums taken block by block (rows through the
+//   block-slot tables), also writing the block means of Q and K: the pooling that the scores
+//   need, from the same pass over Q and K (bsa_problem.block_means).
 // drift_finalize_kernel grid (chunks, heads): every CTA reduces its head's partials in a
 //   fixed order (deterministic), so all of them agree on the decision; CTA 0 publishes
 //   drift/refresh and, for a refreshed head, each CTA copies its chunk of Q, K to the
@@ -97,22 +100,111 @@ __global__ void __launch_bounds__(kDriftThreads) drift_partial_kernel(
     }
 }
 
+// grid (nb, heads), kDriftPoolThreads threads: block i of head h. Query rows come from perm,
+// key rows from kperm (per head, nullable: perm). Each thread owns 16-byte chunk c of NIT rows,
+// taken two rows at a time (eight 16-byte loads of the four tensors in flight per thread, few
+// registers, three CTAs per SM so that one CTA's loads overlap another's stores). Writes the
+// four drift sums of the block (float64, fixed order) to part[h][i] and the means of Q and K
+// over the block's real tokens to qbar/kbar [heads][nb][D]; with force_all also the snapshot
+// (Q -> Qref, K -> Kref).
+constexpr int kDriftPoolThreads = 256;
+
+template <int D, int B>
+__global__ void __launch_bounds__(kDriftPoolThreads, 3) drift_pool_kernel(
+    Geom g, const bsa_bf16* __restrict__ Q, const bsa_bf16* __restrict__ K, bsa_bf16* Qref, bsa_bf16* Kref,
+    const int* __restrict__ perm, const int* __restrict__ kperm, int force_all, double* __restrict__ part,
+    float* __restrict__ qbar, float* __restrict__ kbar) {
+    constexpr int CH = D / 8;                       // 16-byte chunks per row
+    constexpr int RPP = kDriftPoolThreads / CH;     // rows per pass
+    constexpr int NIT = B / RPP;                    // passes
+    constexpr int PH = NIT >= 2 ? 2 : 1;            // rows loaded together
+    static_assert(NIT >= 1 && RPP * NIT == B && NIT % PH == 0, "block rows per thread");
+    const int i = blockIdx.x, h = blockIdx.y;
+    const int c = threadIdx.x % CH, rs = threadIdx.x / CH;
+    const size_t head_off = (size_t)h * g.N * D;
+    const int* kp = kperm != nullptr ? kperm + (size_t)h * g.nb * B : perm;
+    float dq = 0.f, sq = 0.f, dk = 0.f, sk = 0.f;
+    float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int k0 = 0; k0 < NIT; k0 += PH) {
+        uint4 vq[PH], vk[PH], rq[PH], rk[PH];
+        int tq[PH], tk[PH];
+#pragma unroll
+        for (int u = 0; u < PH; ++u) {
+            const int slot = i * B + rs + (k0 + u) * RPP;
+            tq[u] = __ldg(perm + slot);
+            tk[u] = min(__ldg(kp + slot), g.N - 1);
+            const size_t oq = head_off + (size_t)max(tq[u], 0) * D + c * 8;
+            const size_t ok = head_off + (size_t)max(tk[u], 0) * D + c * 8;
+            vq[u] = tq[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(Q + oq)) : z;
+            vk[u] = tk[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(K + ok)) : z;
+            rq[u] = tq[u] >= 0 ? *reinterpret_cast<const uint4*>(Qref + oq) : z;
+            rk[u] = tk[u] >= 0 ? *reinterpret_cast<const uint4*>(Kref + ok) : z;
+        }
+#pragma unroll
+        for (int u = 0; u < PH; ++u) {
+            drift_accum(vq[u], rq[u], dq, sq);
+            drift_accum(vk[u], rk[u], dk, sk);
+            const __nv_bfloat162* pq = reinterpret_cast<const __nv_bfloat162*>(&vq[u]);
+            const __nv_bfloat162* pk = reinterpret_cast<const __nv_bfloat162*>(&vk[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 a = __bfloat1622float2(pq[e]), b = __bfloat1622float2(pk[e]);
+                aq[2 * e] += a.x;
+                aq[2 * e + 1] += a.y;
+                ak[2 * e] += b.x;
+                ak[2 * e + 1] += b.y;
+            }
+            if (force_all) {
+                if (tq[u] >= 0) *reinterpret_cast<uint4*>(Qref + head_off + (size_t)tq[u] * D + c * 8) = vq[u];
+                if (tk[u] >= 0) *reinterpret_cast<uint4*>(Kref + head_off + (size_t)tk[u] * D + c * 8) = vk[u];
+            }
+        }
+    }
+    // block means: the RPP row groups' sums through shared memory, in a fixed order
+    __shared__ float red[2][RPP][D + 4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        red[0][rs][c * 8 + e] = aq[e];
+        red[1][rs][c * 8 + e] = ak[e];
+    }
+    __shared__ double scratch[kDriftPoolThreads / 32];
+    const double s0 = block_sum_double((double)dq, scratch);   // (its first __syncthreads also
+    const double s1 = block_sum_double((double)sq, scratch);   //  orders the stores to red)
+    const double s2 = block_sum_double((double)dk, scratch);
+    const double s3 = block_sum_double((double)sk, scratch);
+    if (threadIdx.x == 0) {
+        double* o = part + ((size_t)h * g.nb + i) * 4;
+        o[0] = s0; o[1] = s1; o[2] = s2; o[3] = s3;
+    }
+    for (int t = threadIdx.x; t < 2 * D; t += kDriftPoolThreads) {
+        const int which = t / D, col = t % D;
+        float s = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < RPP; ++r) s += red[which][r][col];
+        const float n = (float)block_count(g, i);
+        float* out = which == 0 ? qbar : kbar;
+        out[((size_t)h * g.nb + i) * D + col] = s / n;
+    }
+}
+
 __device__ inline double rel_change(double diff2, double ref2) {
     if (ref2 == 0.0) return diff2 == 0.0 ? 0.0 : (double)INFINITY;
     return sqrt(diff2 / ref2);
 }
 
-// grid (chunks or 1, heads): nchunks is the number of partials per head.
+// grid (copy chunks of kDriftChunkElems, or 1 with force_all, heads); nparts partials per head.
 __global__ void __launch_bounds__(kDriftThreads) drift_finalize_kernel(
     const bsa_bf16* __restrict__ Q, const bsa_bf16* __restrict__ K, bsa_bf16* Qref,
     bsa_bf16* Kref, long long elems, int force_all, float tau,
-    const double* __restrict__ part, float* __restrict__ drift, int* __restrict__ refresh, int nchunks) {
+    const double* __restrict__ part, float* __restrict__ drift, int* __restrict__ refresh, int nparts) {
     const int c = blockIdx.x, h = blockIdx.y;
     __shared__ double scratch[kDriftThreads / 32];
     __shared__ int s_refresh;
     double acc[4] = {0, 0, 0, 0};
-    const double* ph = part + (size_t)h * nchunks * 4;
-    for (int k = threadIdx.x; k < nchunks; k += kDriftThreads) {
+    const double* ph = part + (size_t)h * nparts * 4;
+    for (int k = threadIdx.x; k < nparts; k += kDriftThreads) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] += ph[(size_t)k * 4 + e];
     }

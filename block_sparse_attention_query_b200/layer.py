@@ -5,7 +5,8 @@ libbsa, with no host synchronisation.
 `SparseAttentionLayer` — drift-gated mask reuse (HEART abstract, Temporal Mask Reuse; HASTE
 abstract): each step runs
 
-    drift_check -> score_blocks(refreshed heads) -> select_topp(refreshed heads) -> attention
+    drift_check (+ block means) -> score_blocks(refreshed heads) -> select_topp(refreshed heads)
+    -> attention
 
 `OneShotLayer` — one-shot estimate with cached reuse and optional Turbo stages (RAPID English
 abstract): dense attention before the estimate step; at the estimate step every head is
@@ -26,12 +27,16 @@ def _per_head(p, heads):
 class SparseAttentionLayer:
     def __init__(self, heads, d, T, H, W, text_tokens=0, block=128, p=0.9, tau=0.05,
                  score_mode=bsa.BSA_SCORE_MEANPOOL, tile=(0, 0, 0), device="cuda"):
-        self.prob = bsa.problem(heads, d, T, H, W, text_tokens, block, tile, score_mode)
+        plan = bsa.bsa_plan(bsa.problem(heads, d, T, H, W, text_tokens, block, tile, score_mode))
+        dev = torch.device(device)
+        # the drift pass also writes the block means that the scores need (one read of Q, K)
+        self.block_means = torch.empty(2, heads, plan.nb, d, dtype=torch.float32, device=dev)
+        self.prob = bsa.problem(heads, d, T, H, W, text_tokens, block, tile, score_mode,
+                                block_means=self.block_means)
         self.plan = bsa.bsa_plan(self.prob)
         self.heads, self.d, self.N = heads, d, self.prob.tokens
         nb = self.plan.nb
         self.nb = nb
-        dev = torch.device(device)
         self.p = torch.tensor(_per_head(p, heads), dtype=torch.float32, device=dev)
         self.tau = float(tau)
         self.scores = torch.zeros(heads, nb, nb, dtype=torch.float32, device=dev)

@@ -88,6 +88,13 @@ typedef struct bsa_problem {
                                through it; queries always use the tile layout. NULL: keys use
                                the tile layout too. Entries outside [-1, tokens) are clamped
                                into range (a wrong table gives wrong results, never a fault). */
+    float* block_means;     /* DEVICE pointer, nullable: caller-owned [2][heads][nb][d] float32.
+                               When set, bsa_drift_check reads Q, K, Q_ref, K_ref block by block
+                               and also writes the block means of Q (first half) and K (second
+                               half; through key_table when set) over each block's real tokens,
+                               and bsa_score_blocks takes its means from there instead of reading
+                               Q and K again: call them in that order on the same Q, K. NULL: each
+                               call reads what it needs. */
 } bsa_problem;
 
 /* Derived sizes, filled by bsa_plan (host only, no CUDA call). */
@@ -158,7 +165,8 @@ int bsa_select_topp(const bsa_problem* prob, const float* scores, const float* p
  *   Q_ref, K_ref   [heads, tokens, d] bf16, in/out reference snapshots.
  *   drift          [heads] float32 out;  refresh [heads] int32 out (0/1; usable as head_mask).
  *   ws             at least plan.drift_workspace_bytes. The reduction order is fixed, so the
- *                  result is deterministic. */
+ *                  result is deterministic. With prob->block_means set, the same pass also
+ *                  writes the block means (see bsa_problem). */
 int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                     bsa_bf16* Q_ref, bsa_bf16* K_ref, float tau, int force_all,
                     float* drift, int* refresh,
@@ -171,7 +179,8 @@ int bsa_drift_check(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* 
  * and outputs. This entry point takes no workspace and allocates nothing: its scratch is a
  * 2 MiB static device array inside the library (held on every device that loads the library
  * until the process exits).
- *   Arguments, results and determinism are those of bsa_drift_check.
+ *   Arguments, results and determinism are those of bsa_drift_check; prob->block_means is
+ *   ignored (the means are not written).
  *   Limit: heads * ceil(tokens * d / 16384) <= 65536; larger problems return
  *          BSA_ERR_SCRATCH_LIMIT and launch nothing.
  *   The first call on a device looks up the scratch address on that device (make that first

@@ -136,4 +136,13 @@ def test_calls_reject_bad_pointers_before_launch():
     assert L.bsa_score_blocks(pb, a, a, None, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
     assert L.bsa_sparse_attention(pb, a, a, a, a, a, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
     assert L.bsa_captured_mass(pb, a, a, a, a, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
+    # block means: a misaligned buffer is refused by both calls that use it
+    bm = bsa.problem(2, 64, 4, 16, 16, 0, 64)
+    bm.block_means = 4096 + 8
+    pbm = ctypes.byref(bm)
+    dw = bsa.bsa_plan(bm).drift_workspace_bytes
+    assert L.bsa_drift_check(pbm, a, a, a, a, ctypes.c_float(0.05), 0, a, a, a, dw, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_score_blocks(pbm, a, a, None, a, a, 1 << 30, None) == bsa.BSA_ERR_ALIGN
+    bm.block_means = 4096
+    assert L.bsa_drift_check(pbm, a, a, a, a, ctypes.c_float(0.05), 0, a, a, a, dw - 1, None) == bsa.BSA_ERR_WORKSPACE
     assert bsa.bsa_launch_count() == launches_before     # none of the rejected calls launched

@@ -707,3 +707,62 @@ def test_full_size_cluster_keys_sampled():
     for h in (0, c.heads - 1):
         n, _ = _check_clustering(c, h, table[h], assign[h], 2)
         print(f"\n[key clustering] wan13b_480p head {h}: {n} assignments differ from the oracle")
+
+
+# ------------------------------------------------------ drift pass with the block means
+
+@pytest.mark.parametrize("name", ["text_d64_b128", "ragged_d128_b64", "text_d128_b128"])
+@pytest.mark.parametrize("force", [0, 1])
+def test_drift_pass_writes_block_means(name, force):
+    """bsa_problem.block_means set: the drift pass reads Q, K, Q_ref, K_ref block by block and
+    also writes the block means. Drift, refresh flags and snapshots as without it (against the
+    oracle), the means against the oracle's pooling (float32 sums of at most 128 bf16 values,
+    bounded by 64 roundings of the mean absolute value), and the scores computed from them."""
+    bsa = _bsa()
+    c = Case(**SMALL[name])
+    rng = np.random.default_rng(11)
+    scale = np.linspace(1.0, 1.2, c.heads)
+    Q2 = inputs.f32_to_bf16_bits((O.bf16_to_f64(c.Qb) * scale[:, None, None]).astype(np.float32))
+    K2 = c.Kb.copy()
+    K2[-1, :7] = inputs.f32_to_bf16_bits(rng.standard_normal((7, c.d)).astype(np.float32))
+    means = torch.full((2, c.heads, c.nb, c.d), float("nan"), dtype=torch.float32, device="cuda")
+    prob = bsa.problem(c.heads, c.d, *_grid(name), c.B, block_means=means)
+    plan = bsa.bsa_plan(prob)
+    Qd, Kd = PT.to_dev_bf16(Q2), PT.to_dev_bf16(K2)
+    Qr, Kr = PT.to_dev_bf16(c.Qb), PT.to_dev_bf16(c.Kb)
+    drift = torch.zeros(c.heads, dtype=torch.float32, device="cuda")
+    refresh = torch.zeros(c.heads, dtype=torch.int32, device="cuda")
+    bsa.bsa_drift_check(prob, Qd, Kd, Qr, Kr, 0.05, force, drift, refresh, c.ws(plan.drift_workspace_bytes))
+    _status_ok()
+    m = means.cpu().numpy()
+    qr, kr = PT.from_dev_bf16(Qr), PT.from_dev_bf16(Kr)
+    for h in range(c.heads):
+        Qh, Kh = O.bf16_to_f64(Q2[h]), O.bf16_to_f64(K2[h])
+        ref = O.drift(Qh, Kh, O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h]))
+        assert drift[h].item() == pytest.approx(ref, rel=1e-6, abs=1e-9)
+        fresh = bool(force) or ref > 0.05
+        assert bool(refresh[h].item()) == fresh
+        assert np.array_equal(qr[h], Q2[h] if fresh else c.Qb[h])
+        assert np.array_equal(kr[h], K2[h] if fresh else c.Kb[h])
+        for X, got in ((Qh, m[0, h]), (Kh, m[1, h])):
+            exact = O.pool_blocks(X, c.layout)
+            tol = 64 * PT.U32 * O.pool_blocks(np.abs(X), c.layout)
+            assert np.all(np.abs(got - exact) <= tol), (h, float(np.abs(got - exact).max()))
+    # the scores taken from these means equal those of a call that pools Q, K itself
+    S1 = torch.empty(c.heads, c.nb, c.nb, dtype=torch.float32, device="cuda")
+    bsa.bsa_score_blocks(prob, Qd, Kd, None, S1, c.ws(plan.score_workspace_bytes))
+    S2 = torch.empty_like(S1)
+    bsa.bsa_score_blocks(bsa.problem(c.heads, c.d, *_grid(name), c.B), Qd, Kd, None, S2,
+                         c.ws(plan.score_workspace_bytes))
+    _status_ok()
+    for h in range(c.heads):
+        Qh, Kh = O.bf16_to_f64(Q2[h]), O.bf16_to_f64(K2[h])
+        ref = O.score_meanpool(Qh, Kh, c.layout)
+        bnd = PT.score_bound(Qh, Kh, c.layout, "meanpool", ref)
+        _check_scores(S1[h].cpu().numpy(), ref, bnd, ("block means", name, h))
+        _check_scores(S2[h].cpu().numpy(), ref, bnd, ("pooled in the call", name, h))
+
+
+def _grid(name):
+    s = SMALL[name]
+    return s["T"], s["H"], s["W"], s["text"]
