@@ -87,6 +87,7 @@ EXPORTS = {
     "bsa_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_version": (ctypes.c_char_p, []),
     "bsa_launch_count": (ctypes.c_ulonglong, []),
+    "bsa_set_park_kernel": (ctypes.c_int, [ctypes.c_int]),
 }
 
 
@@ -214,3 +215,11 @@ def bsa_version() -> str:
 
 def bsa_launch_count() -> int:
     return int(lib.bsa_launch_count())
+
+
+PARK_AUTO = 0
+PARK_TWO_PASS = 1
+
+
+def bsa_set_park_kernel(which: int) -> int:
+    return lib.bsa_set_park_kernel(which)

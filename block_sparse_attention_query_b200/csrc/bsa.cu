@@ -10,6 +10,7 @@
 #include "bsa_common.cuh"
 #include "score.cuh"
 #include "park_tc.cuh"
+#include "park_cluster.cuh"
 #include "meanpool_tc.cuh"
 #include "select.cuh"
 #include "drift.cuh"
@@ -94,7 +95,29 @@ size_t perm_bytes(const Geom& g) { return align256((size_t)g.nb * g.B * sizeof(i
 
 // Score workspace: [pooled Q means | pooled K means: heads*nb*d fp32 each][block-slot table]
 size_t pooled_bytes(const Geom& g) { return align256((size_t)2 * g.heads * g.nb * g.d * sizeof(float)); }
-int park_nbp(const Geom& g) { return (g.nb + park::NT - 1) / park::NT * park::NT; }
+// bsa_set_park_kernel: BSA_PARK_TWO_PASS forces the two-pass PARK kernel.
+std::atomic<int> g_park_two_pass{0};
+
+int tile_nbp(const Geom& g) { return (g.nb + park::NT - 1) / park::NT * park::NT; }
+// PARK in one pass: key blocks split over a cluster of C CTAs, W per CTA (a multiple of 16);
+// false when nb needs more than the largest portable cluster.
+bool park_cluster_shape(const Geom& g, int* C, int* W) {
+    const int wmax = parkc::kMaxCols;
+    const int c = (g.nb + wmax - 1) / wmax;
+    if (c < 1 || c > parkc::kMaxCluster) return false;
+    const int w = ((g.nb + c - 1) / c + 15) / 16 * 16;
+    if ((c - 1) * w >= g.nb) return false;   // every CTA holds at least one real key block
+    *C = c;
+    *W = w;
+    return true;
+}
+// Rows of each bf16 part of the pooled keys per head: the tile count of the two-pass kernels,
+// or the cluster's C * W, whichever is larger.
+int park_nbp(const Geom& g) {
+    int C = 0, W = 0, n = tile_nbp(g);
+    if (park_cluster_shape(g, &C, &W) && C * W > n) n = (C * W + park::NT - 1) / park::NT * park::NT;
+    return n;
+}
 // Both scorers keep the three bf16 parts of the pooled keys, [heads][3][nbp][d]; the
 // mean-pooled one also those of the pooled queries, [heads][3][nbq][d] (nbq: nb rounded up to
 // a multiple of 128), then one float per score row (its softmax offset).
@@ -107,6 +130,61 @@ size_t score_ws_bytes(const Geom& g, int mode) {
            (mode == BSA_SCORE_MEANPOOL ? qsplit_bytes(g) + rowoff_bytes(g) : 0);
 }
 
+int sm_count();
+
+// One-pass PARK on clusters; BSA_ERR_UNSUPPORTED when the shape or the device leaves it out
+// (the caller then runs the two-pass kernel).
+template <int D>
+int launch_park_cluster(const Geom& g, const bsa_bf16* Q, const int* perm, const int* head_mask, float* scores,
+                        const bsa_bf16* ksplit, int nbp, cudaStream_t st) {
+    int C = 0, W = 0;
+    if (!park_cluster_shape(g, &C, &W) || C * W > nbp) return BSA_ERR_UNSUPPORTED;
+    const parkc::Layout L = parkc::layout<D>(W, C);
+    if (L.total > 232448) return BSA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(parkc::park_cluster_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) !=
+        cudaSuccess)
+        return BSA_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms <= 0) return BSA_ERR_CUDA;
+    parkc::Params P;
+    P.g = g;
+    P.Q = Q;
+    P.ksplit = ksplit;
+    P.perm = perm;
+    P.head_mask = head_mask;
+    P.scores = scores;
+    P.nbp = nbp;
+    P.W = W;
+    P.C = C;
+    P.n_items = g.heads * g.nb;
+    P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sms / C * C));
+    cfg.blockDim = dim3(parkc::kThreads);
+    cfg.dynamicSmemBytes = (size_t)L.total;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, parkc::park_cluster_kernel<D>, &cfg) != cudaSuccess || ncl <= 0) {
+        (void)cudaGetLastError();
+        return BSA_ERR_UNSUPPORTED;
+    }
+    if (ncl > P.n_items) ncl = P.n_items;
+    P.n_clusters = ncl;
+    cfg.gridDim = dim3((unsigned)(ncl * C));
+    if (cudaLaunchKernelEx(&cfg, parkc::park_cluster_kernel<D>, P) != cudaSuccess) {
+        launch_status();
+        return BSA_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 template <int D>
 int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* perm, const int* head_mask,
                 float* scores, bsa_bf16* ksplit, cudaStream_t st) {
@@ -115,6 +193,10 @@ int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* 
     const long long n = (long long)g.heads * nbp * D;
     park::split_kbar_kernel<D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(g, kbar, nbp, ksplit);
     if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
+    if (!g_park_two_pass) {
+        const int rc = launch_park_cluster<D>(g, Q, perm, head_mask, scores, ksplit, nbp, st);
+        if (rc != BSA_ERR_UNSUPPORTED) return rc;
+    }
     if (cudaFuncSetAttribute(park::park_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
         return BSA_ERR_CUDA;
@@ -137,13 +219,11 @@ int launch_park(const Geom& g, const bsa_bf16* Q, const float* kbar, const int* 
     return launch_status();
 }
 
-int sm_count();
-
 template <int D>
 int launch_meanpool(const Geom& g, const float* qbar, const float* kbar, const int* head_mask, float* scores,
                     bsa_bf16* qsplit, bsa_bf16* ksplit, float* rowoff, cudaStream_t st) {
     using C = mp::Cfg<D>;
-    const int nbq = mp_nbq(g), nbp = park_nbp(g);
+    const int nbq = mp_nbq(g), nbp = tile_nbp(g);
     const long long nq = (long long)g.heads * nbq * D, nk = (long long)g.heads * nbp * D;
     park::split_kbar_kernel<D><<<(unsigned)((nq + 255) / 256), 256, 0, st>>>(g, qbar, nbq, qsplit);
     if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
@@ -706,6 +786,12 @@ const char* bsa_error_string(int status) {
 }
 
 const char* bsa_version(void) { return "bsa 0.2.0 sm_100a"; }
+
+int bsa_set_park_kernel(int which) {
+    if (which != BSA_PARK_AUTO && which != BSA_PARK_TWO_PASS) return BSA_ERR_ARG;
+    g_park_two_pass.store(which == BSA_PARK_TWO_PASS ? 1 : 0);
+    return BSA_OK;
+}
 
 unsigned long long bsa_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 

@@ -172,6 +172,61 @@ __device__ inline uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
+// ----------------------------------------------------------- PTX: thread-block clusters
+
+__device__ inline uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address in CTA `rank`'s shared memory of the object at `addr` in this CTA's (same offset).
+__device__ inline uint32_t cluster_map(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Asynchronous 8-byte store into another CTA's shared memory; on arrival it counts its bytes
+// against that CTA's mbarrier `cluster_bar` (complete_tx). The issuing thread does not wait.
+__device__ inline void st_async_f32x2(uint32_t cluster_addr, float a, float b, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 ::"r"(cluster_addr), "f"(a), "f"(b), "r"(cluster_bar) : "memory");
+}
+
+// Arrive on a local mbarrier and raise the bytes its current phase waits for.
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// try_wait with cluster-scope acquire: what other CTAs of the cluster wrote before their
+// arrivals (or stored with complete_tx on this barrier) is visible once it returns true.
+__device__ inline bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u) : "memory");
+    return ok != 0;
+}
+
+// mbar_wait for a barrier that other CTAs of the cluster arrive on.
+__device__ inline bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned epoch) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (timed_out_since(epoch)) return false;
+        if (clock64() - t0 > kWaitLimitCycles) { raise_timeout(); return false; }
+    }
+    return true;
+}
+
+// Every thread of every CTA of the cluster (all of them must execute it).
+__device__ inline void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ PTX: cp.async
 
 __device__ inline void cp_async_16(uint32_t dst_smem, const void* src) {

@@ -43,7 +43,8 @@ struct Cfg {
     static constexpr int OFF_Q = 0;                          // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // NS stages of 3 splits
     static constexpr int OFF_COL = OFF_K + NS * STAGE_BYTES; // [2][4 warps][NT] column sums
-    static constexpr int OFF_BAR = OFF_COL + 2 * 4 * NT * 4;
+    static constexpr int OFF_TOK = OFF_COL + 2 * 4 * NT * 4;  // [2 loader warps][BQ] int: query-tile tokens
+    static constexpr int OFF_BAR = OFF_TOK + 2 * BQ * 4;
     // q_full[2] q_empty[2] k_full[NS] k_empty[NS] l_full[2] l_free[2] col[1] fin
     static constexpr int NBAR = 4 + 2 * NS + 4 + 1 + 1;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 8;
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
     uint64_t* fin_bar = col_bar + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + C::NBAR * 8);
     float* colpart = reinterpret_cast<float*>(sm + C::OFF_COL);
+    int* qtok = reinterpret_cast<int*>(sm + C::OFF_TOK);
 
     const Geom& g = P.g;
     const int warp = threadIdx.x >> 5;
@@ -162,21 +164,31 @@ __global__ void __launch_bounds__(kThreads, 1) park_tc_kernel(Params P) {
             if (skip_item(item)) continue;
             const int h = item / nb, i = item - h * nb;
             const int qb = k & 1;
-            if (k >= 2) ok = mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch);
+            // loader waits are warp-uniform (__all_sync): the warp syncs below need every lane
+            if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[qb], ((k >> 1) - 1) & 1, epoch));
             if (!ok) break;
             const bsa_bf16* Qh = P.Q + (size_t)h * g.N * D;
-            const int* slot = P.perm + i * g.B;
-            for (int r = lt / CH; r < BQ; r += kLoadThreads / CH) {
-                int tok = r < g.B ? __ldg(slot + r) : -1;
-                if (tok < 0) tok = 0;
-                cp_async_16(sQ + qb * C::Q_BYTES + sw128_offset(BQ, r, c), Qh + (size_t)tok * D + c * 8);
+            // the tile's tokens: one coalesced load per loader warp into its own copy in shared
+            // memory, then the row gathers (no gather waits on a load of its own token)
+            {
+                int* wtok = qtok + (lt >> 5) * BQ;
+                const int ln = lt & 31;
+                int4 t4 = make_int4(-1, -1, -1, -1);
+                if (4 * ln < g.B) t4 = __ldg(reinterpret_cast<const int4*>(P.perm + (size_t)i * g.B) + ln);
+                reinterpret_cast<int4*>(wtok)[ln] = t4;
+                __syncwarp();
+                for (int r = lt / CH; r < BQ; r += kLoadThreads / CH) {
+                    const int tok = max(wtok[r], 0);
+                    cp_async_16(sQ + qb * C::Q_BYTES + sw128_offset(BQ, r, c), Qh + (size_t)tok * D + c * 8);
+                }
+                __syncwarp();                            // the copy is rewritten for the next item
             }
             cp_async_arrive_noinc(&q_full[qb]);
             const bsa_bf16* kh = P.ksplit + (size_t)h * 3 * P.nbp * D;
             for (int t2 = 0; t2 < 2 * ntiles && ok; ++t2, ++gt) {
                 const int t = t2 % ntiles;                   // pass A tiles, then pass B tiles
                 const int s = gt % NS;
-                if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1, epoch);
+                if (gt >= NS) ok = __all_sync(0xffffffffu, mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1, epoch));
                 if (!ok) break;
 #pragma unroll
                 for (int sp = 0; sp < 3; ++sp) {

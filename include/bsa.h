@@ -133,7 +133,8 @@ int bsa_block_layout(const bsa_problem* prob, int* perm_host);
  *              size depends on the mode, so plan with the mode that will run.
  * Mode is prob->score_mode. Mean-pooled scores are float32-grade: float32 dot products on
  * CUDA cores for problems too small to fill the GPU, otherwise tensor-core products of the
- * bf16 splits; both agree with exact arithmetic to float32 rounding. */
+ * bf16 splits; both agree with exact arithmetic to float32 rounding. PARK scores are
+ * float32-grade too, from one of two tensor-core kernels (bsa_set_park_kernel). */
 int bsa_score_blocks(const bsa_problem* prob, const bsa_bf16* Q, const bsa_bf16* K,
                      const int* head_mask, float* scores,
                      void* ws, size_t ws_bytes, bsa_stream_t stream);
@@ -273,6 +274,18 @@ int bsa_device_status(bsa_stream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* bsa_error_string(int status);
+
+/* Which kernel bsa_score_blocks runs in PARK mode (process-wide host setting, no CUDA call;
+ * takes effect at the next call):
+ *   BSA_PARK_AUTO      one pass, each item's logits held in tensor memory, the key blocks of
+ *                      a head split over a thread-block cluster of up to 8 CTAs (nb up to
+ *                      1280); larger nb, or a device that cannot place the cluster, falls
+ *                      back to the two-pass kernel. The default.
+ *   BSA_PARK_TWO_PASS  always the two-pass kernel (64-block tiles, logits computed twice).
+ * Both give the same scores to float32 rounding. Returns BSA_OK or BSA_ERR_ARG. */
+#define BSA_PARK_AUTO     0
+#define BSA_PARK_TWO_PASS 1
+int bsa_set_park_kernel(int which);
 
 /* Library version, e.g. "bsa 0.2.0 sm_100a". */
 const char* bsa_version(void);

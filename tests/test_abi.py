@@ -32,6 +32,14 @@ def test_exports_every_declared_symbol():
         assert n in bsa.EXPORTS, n
 
 
+def test_park_kernel_setting_is_checked_on_the_host():
+    # a process-wide host setting: no CUDA call, so it runs without a GPU
+    assert bsa.bsa_set_park_kernel(bsa.PARK_TWO_PASS) == 0
+    assert bsa.bsa_set_park_kernel(2) == bsa.BSA_ERR_ARG
+    assert bsa.bsa_set_park_kernel(-1) == bsa.BSA_ERR_ARG
+    assert bsa.bsa_set_park_kernel(bsa.PARK_AUTO) == 0
+
+
 def test_version_and_error_strings():
     assert "sm_100a" in bsa.bsa_version()
     for code in range(-7, 1):

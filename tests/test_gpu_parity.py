@@ -151,6 +151,40 @@ def test_scores_tensor_core_path_match_oracle(name):
         _check_scores(S[h], ref, bnd, (name, h))
 
 
+# PARK's one-pass kernel with the key blocks of a head split over a cluster of CTAs: nb above
+# one CTA's share (176 key blocks for d = 128, 256 for d = 64), a partial last chunk, text
+# blocks. The two-pass kernel runs on the same inputs, and a masked head stays untouched.
+PARK_CLUSTER = {
+    "c3_d128_b64_text": dict(heads=2, d=128, T=8, H=48, W=60, text=100, B=64, p=0.9),   # nb 362: 3 x 128
+    "c2_d64_b64": dict(heads=2, d=64, T=9, H=32, W=60, text=0, B=64, p=0.9),             # nb 270: 2 x 144
+}
+
+
+@pytest.mark.parametrize("name", list(PARK_CLUSTER))
+def test_park_cluster_kernel_matches_oracle_and_two_pass(name):
+    bsa = _bsa()
+    c = Case(**PARK_CLUSTER[name], mode="park")
+    S1 = c.gpu_scores()
+    try:
+        assert bsa.bsa_set_park_kernel(bsa.PARK_TWO_PASS) == 0
+        S2 = c.gpu_scores()
+    finally:
+        assert bsa.bsa_set_park_kernel(bsa.PARK_AUTO) == 0
+    mask = torch.ones(c.heads, dtype=torch.int32, device="cuda")
+    mask[1] = 0
+    S3 = torch.full_like(S1, -1.0)
+    bsa.bsa_score_blocks(c.prob, c.Q, c.K, mask, S3, c.ws(c.plan.score_workspace_bytes))
+    torch.cuda.synchronize()
+    _status_ok()
+    assert (S3[1] == -1.0).all()
+    assert torch.equal(S3[0], S1[0])          # same kernel, same inputs: the same bits
+    S1, S2 = S1.cpu().numpy(), S2.cpu().numpy()
+    for h in range(c.heads):
+        ref, bnd = c.oracle_scores_and_bound(h)
+        _check_scores(S1[h], ref, bnd, (name, "one-pass", h))
+        _check_scores(S2[h], ref, bnd, (name, "two-pass", h))
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_select_on_oracle_scores_is_exact(name):
     # same float32 scores on both sides: only the cumulative-sum rounding may differ
