@@ -97,6 +97,70 @@ __device__ inline float ex2(float x) {
     return y;
 }
 
+// Pass A over NC consecutive 32-column chunks of a row (tcgen05 loads in flight together); the
+// last chunk holds `nv_last` real columns (the rest is masked to -inf). Updates the running max
+// mt (scaled logits) and the sum lt of 2^(x - mt); writes 2^(x - mn) back (mn = the new
+// running max, returned as the chunks' reference).
+template <int NC>
+__device__ inline float pass_a_chunks(uint32_t taddr, int nv_last, float sc, float& mt, float& lt) {
+    uint32_t v[NC][32];
+#pragma unroll
+    for (int u = 0; u < NC; ++u) tmem_ld32(taddr + u * 32, v[u]);
+    tmem_wait_ld();
+    if (nv_last < 32) {                                  // warp-uniform: only a row's last chunk
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (e >= nv_last) v[NC - 1][e] = __float_as_uint(-INFINITY);
+    }
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int u = 0; u < NC; ++u)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[u][e]));
+    const float mn = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc);
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < NC; ++u) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const float x = ex2(fmaf(__uint_as_float(v[u][e]), sc, -mn));   // -inf -> 0
+            ls[e & 3] += x;
+            v[u][e] = __float_as_uint(x);
+        }
+        tmem_st32(taddr + u * 32, v[u]);
+    }
+    lt = lt * ex2(mt - mn) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));   // the first chunks: 0 * 0
+    mt = mn;
+    return mn;
+}
+
+// Pass B over NC consecutive chunks: p = e * f summed over the warp's 32 rows (transpose-reduce:
+// after five halvings lane l holds column l's sum), written to col[u * 32 + lane].
+template <int NC>
+__device__ inline void pass_b_chunks(uint32_t taddr, float f, int lane, float* col) {
+    uint32_t v[NC][32];
+#pragma unroll
+    for (int u = 0; u < NC; ++u) tmem_ld32(taddr + u * 32, v[u]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < NC; ++u) {
+        uint32_t* p = v[u];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) p[e] = __float_as_uint(__uint_as_float(p[e]) * f);
+#pragma unroll
+        for (int o = 16, m = 32; o > 0; o >>= 1, m >>= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int e = 0; e < m / 2; ++e) {
+                const float send = __uint_as_float(upper ? p[e] : p[e + m / 2]);
+                const float keep = __uint_as_float(upper ? p[e + m / 2] : p[e]);
+                p[e] = __float_as_uint(keep + __shfl_xor_sync(0xffffffffu, send, o));
+            }
+        }
+        col[u * 32 + lane] = __uint_as_float(p[0]);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -161,9 +225,18 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
     const uint32_t sQ = smem_u32(sm + L.off_q);
     constexpr uint32_t Q_BYTES = BQ * D * 2;
 
+    // masked heads are skipped; the mask of the last head looked at is kept (items come in
+    // head order, so the mask is read about once per head and thread)
+    int mask_h = -1;
+    bool mask_skip = false;
     auto skip_item = [&](long long item) -> bool {
+        if (P.head_mask == nullptr) return false;
         const int h = (int)(item / nb);
-        return P.head_mask != nullptr && P.head_mask[h] == 0;
+        if (h != mask_h) {
+            mask_h = h;
+            mask_skip = P.head_mask[h] == 0;
+        }
+        return mask_skip;
     };
 
     if (warp >= kLoadWarp0) {
@@ -297,7 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
         }
         bool ok = true;
         int n = 0;                                       // this team's item count
-        for (; item >= 0 && ok; item = team_next(item), ++n) {
+        for (long long nx; item >= 0 && ok; item = nx, ++n) {
+            nx = team_next(item);                        // this team's next item, -1 at the end
             const int h = (int)(item / nb), i = (int)(item - (long long)h * nb);
             const bool row_real = r < g.B && __ldg(P.perm + (size_t)i * g.B + r) >= 0;
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[team], n & 1, epoch));
@@ -308,41 +382,16 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
             // running max of their pair (ref), are written back over the logits
             float mt = -INFINITY, lt = 0.f;
             float ref[kGroups];
+#pragma unroll 1
+            for (int gi = 0; gi * kGroup < nch; ++gi) {
+                const int ch = gi * kGroup;
+                const uint32_t ta = tb + ch * 32;
+                float rf;
+                if (ch + 1 < nch) rf = pass_a_chunks<2>(ta, min(32, Wc - (ch + 1) * 32), sc, mt, lt);
+                else rf = pass_a_chunks<1>(ta, min(32, Wc - ch * 32), sc, mt, lt);
 #pragma unroll
-            for (int gi = 0; gi < kGroups; ++gi) {
-                ref[gi] = -INFINITY;
-                if (gi * kGroup >= nch) continue;        // warp-uniform
-                uint32_t v[kGroup][32];
-#pragma unroll
-                for (int u = 0; u < kGroup; ++u)
-                    if (gi * kGroup + u < nch) tmem_ld32(tb + (gi * kGroup + u) * 32, v[u]);
-                tmem_wait_ld();
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int u = 0; u < kGroup; ++u) {
-                    const int ch = gi * kGroup + u;
-                    const int nvalid = ch < nch ? min(32, Wc - ch * 32) : 0;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (e < nvalid) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[u][e]));
-                }
-                const float mn = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc);
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int u = 0; u < kGroup; ++u) {
-                    const int ch = gi * kGroup + u;
-                    const int nvalid = ch < nch ? min(32, Wc - ch * 32) : 0;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = e < nvalid ? ex2(fmaf(__uint_as_float(v[u][e]), sc, -mn)) : 0.f;
-                        ls[e & 3] += x;
-                        v[u][e] = __float_as_uint(x);
-                    }
-                    if (ch < nch) tmem_st32(tb + ch * 32, v[u]);
-                }
-                lt = lt * ex2(mt - mn) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));   // the first pair: 0 * 0
-                mt = mn;
-                ref[gi] = mn;
+                for (int q = 0; q < kGroups; ++q)
+                    if (q == gi) ref[q] = rf;                // registers, not local memory
             }
             tmem_wait_st();
             // exchange: this row's (m, l) over the CTA's key blocks, into every CTA of the cluster
@@ -353,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
                 for (int c2 = 0; c2 < C; ++c2)
                     st_async_f32x2(cluster_map(slot, (uint32_t)c2), mt, lt, cluster_map(bar, (uint32_t)c2));
             }
-            if (tt == 0 && team_next(item) >= 0) {
+            if (tt == 0 && nx >= 0) {
                 // the team's next item uses the other barrier, whose previous phase (the team's
                 // item n - 1) was waited on during that item
                 mbar_arrive_expect_tx(&st_full[team * 2 + ((n + 1) & 1)], xbytes);
@@ -371,40 +420,19 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
                 if (s2.y > 0.f) lg += s2.y * ex2(s2.x - mg);
             }
             // pass B: probabilities, summed over the warp's 32 rows per column
+#pragma unroll 1
+            for (int gi = 0; gi * kGroup < nch; ++gi) {
+                const int ch = gi * kGroup;
+                float rf = ref[0];
 #pragma unroll
-            for (int gi = 0; gi < kGroups; ++gi) {
-                if (gi * kGroup >= nch) continue;        // warp-uniform
-                const float f = (row_real && lg > 0.f) ? ex2(ref[gi] - mg) / lg : 0.f;
-                uint32_t v[kGroup][32];
-#pragma unroll
-                for (int u = 0; u < kGroup; ++u)
-                    if (gi * kGroup + u < nch) tmem_ld32(tb + (gi * kGroup + u) * 32, v[u]);
-                tmem_wait_ld();
-                if ((gi + 1) * kGroup >= nch) {
-                    tc_fence_before();
-                    mbar_arrive(&s_free[team]);          // TMEM buffer read for this item
-                }
-#pragma unroll
-                for (int u = 0; u < kGroup; ++u) {
-                    const int ch = gi * kGroup + u;
-                    if (ch >= nch) continue;             // warp-uniform
-                    // warp transpose-reduce of p = e * f: after five halvings lane l holds column l's sum
-                    uint32_t* p = v[u];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) p[e] = __float_as_uint(__uint_as_float(p[e]) * f);
-#pragma unroll
-                    for (int o = 16, m = 32; o > 0; o >>= 1, m >>= 1) {
-                        const bool upper = (lane & o) != 0;
-#pragma unroll
-                        for (int e = 0; e < m / 2; ++e) {
-                            const float send = __uint_as_float(upper ? p[e] : p[e + m / 2]);
-                            const float keep = __uint_as_float(upper ? p[e + m / 2] : p[e]);
-                            p[e] = __float_as_uint(keep + __shfl_xor_sync(0xffffffffu, send, o));
-                        }
-                    }
-                    csum[q4 * kMaxCols + ch * 32 + lane] = __uint_as_float(p[0]);
-                }
+                for (int q = 1; q < kGroups; ++q)
+                    if (q == gi) rf = ref[q];
+                const float f = (row_real && lg > 0.f) ? ex2(rf - mg) / lg : 0.f;
+                if (ch + 1 < nch) pass_b_chunks<2>(tb + ch * 32, f, lane, csum + q4 * kMaxCols + ch * 32);
+                else pass_b_chunks<1>(tb + ch * 32, f, lane, csum + q4 * kMaxCols + ch * 32);
             }
+            tc_fence_before();
+            mbar_arrive(&s_free[team]);                  // TMEM buffer read for this item
             mbar_arrive(&col_bar[team]);
             ok = __all_sync(0xffffffffu, mbar_wait(&col_bar[team], n & 1, epoch));
             if (!ok) break;
