@@ -10,9 +10,9 @@
 // passes over the key tiles, the key blocks of a head are split over a cluster of C CTAs. CTA c
 // keeps the three parts of its W pooled keys (key blocks [cW, cW + W)) resident in shared
 // memory while the cluster works on that head, and per item (head, query block) issues one
-// M = 128, N = W product per part and K step. The 128 x W logits stay in TMEM, in one of two
-// buffers; two softmax teams take the items alternately, one per buffer, so one team's
-// exponentials, the other's column sums and the next item's products overlap:
+// M = 128, N = W product per part and K step. The 128 x W logits stay in TMEM, in one of three
+// buffers used in turn; two softmax teams take the items alternately, so one team's
+// exponentials, the other's column sums and the next items' products overlap:
 //   pass A   per row, in one thread (two 32-column chunks loaded at a time): the running max
 //            m_t and sum l_t of 2^(x - m_t); the exponentials, relative to the running max of
 //            their pair, are written back over the logits;
@@ -42,13 +42,13 @@ constexpr int kLoadWarps = 3;            // a cp.async gather warp moves ~5 B pe
 constexpr int kLoadThreads = 32 * kLoadWarps;
 constexpr int kThreads = 2 * kTeamThreads + 32 + kLoadThreads;   // 384
 constexpr int kMaxCluster = 8;
-constexpr int kBufCols = 256;     // TMEM columns per logit buffer
+constexpr int kBufs = 3;          // TMEM logit buffers, used in turn by consecutive items
 constexpr int kTmemCols = 512;
-constexpr int kNumBars = 17;
+constexpr int kNumBars = 19;
 
 // Most key blocks one CTA holds (five chunks of 32 per row; for d = 128 the three parts of 160
 // pooled keys take 120 KB of shared memory).
-constexpr int kMaxCols = 160;
+constexpr int kMaxCols = 160;     // also the TMEM buffer stride: 3 x 160 columns of the 512
 constexpr int kChunks = kMaxCols / 32;
 constexpr int kGroup = 2;                                   // chunks loaded together
 constexpr int kGroups = (kChunks + kGroup - 1) / kGroup;
@@ -176,11 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
     uint64_t* q_empty = bars + 2;     // [2] query tile read by the products (commit)
     uint64_t* kb_full = bars + 4;     // resident pooled keys landed (loaders)
     uint64_t* kb_free = bars + 5;     // last product of a head done (commit)
-    uint64_t* s_full = bars + 6;      // [2] logits in TMEM buffer (commit)
-    uint64_t* s_free = bars + 8;      // [2] TMEM buffer read for the last time (softmax team)
-    uint64_t* st_full = bars + 10;    // [2 teams][2] the cluster's (m, l) pairs landed (st.async bytes)
-    uint64_t* col_bar = bars + 14;    // [2 teams] the four lane quarters' column sums written
-    uint64_t* fin_bar = bars + 16;
+    uint64_t* s_full = bars + 6;      // [3] logits in TMEM buffer (commit)
+    uint64_t* s_free = bars + 9;      // [3] TMEM buffer read for the last time (softmax team)
+    uint64_t* st_full = bars + 12;    // [2 teams][2] the cluster's (m, l) pairs landed (st.async bytes)
+    uint64_t* col_bar = bars + 16;    // [2 teams] the four lane quarters' column sums written
+    uint64_t* fin_bar = bars + 18;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     float* colsum = reinterpret_cast<float*>(sm + L.off_col);
     float2* stats = reinterpret_cast<float2*>(sm + L.off_stats);
@@ -202,9 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(&q_full[b], kLoadThreads);
             mbar_init(&q_empty[b], 1);
+            mbar_init(&col_bar[b], kTeamThreads);
+        }
+        for (int b = 0; b < kBufs; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&s_free[b], kTeamThreads);
-            mbar_init(&col_bar[b], kTeamThreads);
         }
         for (int b = 0; b < 4; ++b) mbar_init(&st_full[b], 1);   // the local expect_tx arrival; bytes from the peers
         mbar_init(kb_full, kLoadThreads);
@@ -312,9 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
                     prev_h = h;
                     if (!ok) break;
                 }
-                const int qb = k & 1, sb = k & 1;
+                const int qb = k & 1, sb = k % kBufs, su = k / kBufs;   // buffer sb, its use su
                 ok = mbar_wait(&q_full[qb], (k >> 1) & 1, epoch);
-                if (ok && k >= 2) ok = mbar_wait(&s_free[sb], ((k >> 1) - 1) & 1, epoch);
+                if (ok && su >= 1) ok = mbar_wait(&s_free[sb], (su - 1) & 1, epoch);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t qbase = sQ + qb * Q_BYTES;
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = smem_desc_sw128(qbase + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024);
                         const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * (W * 128) + (kk & 3) * 32, 16, 1024);
-                        mma_bf16_ss(tmem + sb * kBufCols, a, b, idesc, (sp < 2 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ss(tmem + sb * kMaxCols, a, b, idesc, (sp < 2 || kk > 0) ? 1u : 0u);
                     }
                 }
                 tc_commit(&s_full[sb]);
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
         const int lane = threadIdx.x & 31;
         const int r = q4 * 32 + lane;                    // query row == TMEM lane
         const int tt = threadIdx.x & (kTeamThreads - 1);
-        const uint32_t tb = tmem + ((uint32_t)(q4 * 32) << 16) + team * kBufCols;   // this team's buffer
+        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);   // this warp's lane quarter
         const float sc = P.scale_log2;
         const uint32_t xbytes = (uint32_t)(C * BQ * 8);  // (m, l) pairs one CTA receives per item
         float* csum = colsum + team * 4 * kMaxCols;
@@ -374,7 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
             nx = team_next(item);                        // this team's next item, -1 at the end
             const int h = (int)(item / nb), i = (int)(item - (long long)h * nb);
             const bool row_real = r < g.B && __ldg(P.perm + (size_t)i * g.B + r) >= 0;
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[team], n & 1, epoch));
+            const int k = 2 * n + team, sb = k % kBufs;  // the CTA's item index, its TMEM buffer
+            const uint32_t tb = tl + sb * kMaxCols;
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (k / kBufs) & 1, epoch));
             if (!ok) break;
             tc_fence_after();
             // pass A: the row's logits, two chunks of 32 at a time (both loads in flight): the
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) park_cluster_kernel(Params P) {
                 else pass_b_chunks<1>(tb + ch * 32, f, lane, csum + q4 * kMaxCols + ch * 32);
             }
             tc_fence_before();
-            mbar_arrive(&s_free[team]);                  // TMEM buffer read for this item
+            mbar_arrive(&s_free[sb]);                    // TMEM buffer read for this item
             mbar_arrive(&col_bar[team]);
             ok = __all_sync(0xffffffffu, mbar_wait(&col_bar[team], n & 1, epoch));
             if (!ok) break;
