@@ -97,6 +97,34 @@ __device__ inline float ex2(float x) {
     return y;
 }
 
+// Packed float32 pairs: one fma.rn.f32x2 / add.rn.f32x2 does both lanes (each lane rounds as
+// the scalar instruction would).
+__device__ inline unsigned long long pk2(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ inline float2 up2(unsigned long long r) {
+    float2 v;
+    asm("mov.b64 {%0,%1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ inline unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ inline unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ inline float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Pass A over NC consecutive 32-column chunks of a row (tcgen05 loads in flight together); the
 // last chunk holds `nv_last` real columns (the rest is masked to -inf). Updates the running max
 // mt (scaled logits) and the sum lt of 2^(x - mt); writes 2^(x - mn) back (mn = the new
@@ -116,20 +144,25 @@ __device__ inline float pass_a_chunks(uint32_t taddr, int nv_last, float sc, flo
 #pragma unroll
     for (int u = 0; u < NC; ++u)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[u][e]));
+        for (int e = 0; e < 32; e += 2)
+            mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], __uint_as_float(v[u][e]), __uint_as_float(v[u][e + 1]));
     const float mn = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc);
-    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+    const unsigned long long sc2 = pk2(sc, sc), neg2 = pk2(-mn, -mn);
+    unsigned long long ls[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
 #pragma unroll
     for (int u = 0; u < NC; ++u) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const float x = ex2(fmaf(__uint_as_float(v[u][e]), sc, -mn));   // -inf -> 0
-            ls[e & 3] += x;
-            v[u][e] = __float_as_uint(x);
+        for (int e = 0; e < 32; e += 2) {
+            const float2 x = up2(fma2(pk2(__uint_as_float(v[u][e]), __uint_as_float(v[u][e + 1])), sc2, neg2));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);                   // -inf -> 0
+            ls[(e >> 1) & 1] = add2(ls[(e >> 1) & 1], pk2(p0, p1));
+            v[u][e] = __float_as_uint(p0);
+            v[u][e + 1] = __float_as_uint(p1);
         }
         tmem_st32(taddr + u * 32, v[u]);
     }
-    lt = lt * ex2(mt - mn) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));   // the first chunks: 0 * 0
+    const float2 l2 = up2(add2(ls[0], ls[1]));
+    lt = lt * ex2(mt - mn) + (l2.x + l2.y);              // the first chunks: 0 * 0
     mt = mn;
     return mn;
 }
@@ -142,22 +175,35 @@ __device__ inline void pass_b_chunks(uint32_t taddr, float f, int lane, float* c
 #pragma unroll
     for (int u = 0; u < NC; ++u) tmem_ld32(taddr + u * 32, v[u]);
     tmem_wait_ld();
+    const unsigned long long f2 = pk2(f, f), zero2 = pk2(0.f, 0.f);
 #pragma unroll
     for (int u = 0; u < NC; ++u) {
-        uint32_t* p = v[u];
+        float p[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) p[e] = __float_as_uint(__uint_as_float(p[e]) * f);
+        for (int e = 0; e < 32; e += 2) {
+            const float2 y = up2(fma2(pk2(__uint_as_float(v[u][e]), __uint_as_float(v[u][e + 1])), f2, zero2));
+            p[e] = y.x;
+            p[e + 1] = y.y;
+        }
 #pragma unroll
-        for (int o = 16, m = 32; o > 0; o >>= 1, m >>= 1) {
+        for (int o = 16, m = 32; o > 1; o >>= 1, m >>= 1) {
             const bool upper = (lane & o) != 0;
 #pragma unroll
-            for (int e = 0; e < m / 2; ++e) {
-                const float send = __uint_as_float(upper ? p[e] : p[e + m / 2]);
-                const float keep = __uint_as_float(upper ? p[e + m / 2] : p[e]);
-                p[e] = __float_as_uint(keep + __shfl_xor_sync(0xffffffffu, send, o));
+            for (int e = 0; e < m / 2; e += 2) {
+                const float s0 = upper ? p[e] : p[e + m / 2], s1 = upper ? p[e + 1] : p[e + 1 + m / 2];
+                const float k0 = upper ? p[e + m / 2] : p[e], k1 = upper ? p[e + 1 + m / 2] : p[e + 1];
+                const float r0 = __shfl_xor_sync(0xffffffffu, s0, o), r1 = __shfl_xor_sync(0xffffffffu, s1, o);
+                const float2 y = up2(add2(pk2(k0, k1), pk2(r0, r1)));
+                p[e] = y.x;
+                p[e + 1] = y.y;
             }
         }
-        col[u * 32 + lane] = __uint_as_float(p[0]);
+        {   // the last halving (offset 1): one column left per lane
+            const bool upper = (lane & 1) != 0;
+            const float sd = upper ? p[0] : p[1], kp = upper ? p[1] : p[0];
+            p[0] = kp + __shfl_xor_sync(0xffffffffu, sd, 1);
+        }
+        col[u * 32 + lane] = p[0];
     }
 }
 
