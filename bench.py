@@ -140,10 +140,11 @@ def _sources_hash(root):
     return hashlib.sha256(src).hexdigest()[:16]
 
 
-def _profiled_traffic(kernel, workload, root=None):
+def _profiled_traffic(kernel, workload, root=None, mode="meanpool"):
     """DRAM bytes per launch of the attention kernel from the committed ncu figures
     (profiles/sparse_attention_<workload>.json), or None when the kernel sources changed since
-    that capture or no capture exists for the workload."""
+    that capture, no capture exists for the workload, or the capture ran another scorer's masks
+    (the traffic follows the kept blocks)."""
     if kernel != "sparse_attention":
         return None
     root = root or os.path.dirname(os.path.abspath(__file__))
@@ -153,6 +154,8 @@ def _profiled_traffic(kernel, workload, root=None):
     with open(prof) as f:
         fields = json.load(f)
     if fields.get("workload") != workload or fields.get("sources_sha256_16") != _sources_hash(root):
+        return None
+    if fields.get("score_mode", "meanpool") != mode:
         return None
     return int(fields["traffic_bytes_per_launch"])
 
@@ -310,7 +313,7 @@ def run_ours(args, ws, rank, local):
         b = bytes_drift if dom == "drift_check" else bytes_score
         ach = b * per_gpu / (stage_ms[names.index(dom)] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4)}
-    traffic = args.traffic if args.traffic is not None else (_profiled_traffic(dom, w.name) if ws == 1 and not args.heads else None)
+    traffic = args.traffic if args.traffic is not None else (_profiled_traffic(dom, w.name, mode=args.mode) if ws == 1 and not args.heads else None)
     roof.update({"kernel": dom,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else peak_src,
                  "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",

@@ -65,6 +65,8 @@ def test_profiled_traffic_only_for_matching_sources(tmp_path):
         json.dump(rec, f)
     assert copy._profiled_traffic("sparse_attention", "hunyuan_720p") == 123456789
     assert copy._profiled_traffic("sparse_attention", "wan13b_480p") is None
+    # the traffic follows the kept blocks: a capture of mean-pooled masks says nothing of PARK's
+    assert copy._profiled_traffic("sparse_attention", "hunyuan_720p", mode="park") is None
     # one byte more in a kernel source: the figure is stale and is not used
     with open(tmp_path / csrc / "attention.cuh", "a") as f:
         f.write("\n")
