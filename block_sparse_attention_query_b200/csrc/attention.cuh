@@ -8,7 +8,7 @@
 // log2-sum-exp) go to the workspace and are merged by merge_text_kernel. Text items come
 // first in the item order, so the long ones start early.
 //
-// Warp roles (480 threads):
+// Warp roles (512 threads):
 //   warps 0-7  softmax, two groups of four warps. Group G takes the blocks g of the stream
 //              with g%2 == G, so the two groups work on consecutive blocks at the same time
 //              (one in its exponentials while the other reads and reduces its scores);
@@ -19,7 +19,7 @@
 //              TMEM, divide by the row sum and store the rows (bf16 O, or the text rows'
 //              float32 partials); also writes the rows of items with nothing kept.
 //   warp 12    TMEM allocation; one elected thread issues every tcgen05.mma.
-//   warps 13-14 loaders: gather Q / K / V rows of a block (raster rows from the block-slot
+//   warps 13-15 loaders: gather Q / K / V rows of a block (raster rows from the block-slot
 //              table) with 16-byte cp.async into 128B-swizzled K-major tiles; completion
 //              arrives on the tile's mbarrier asynchronously.
 // The kept blocks of all items of a CTA form one stream g = 0, 1, 2, ...:
@@ -47,8 +47,8 @@ constexpr int kEpiWarp0 = 8;
 constexpr int kEpiThreads = 128;
 constexpr int kMmaWarp = 12;
 constexpr int kLoadWarp0 = 13;
-constexpr int kLoadThreads = 64;
-constexpr int kThreads = kSoftmaxThreads + kEpiThreads + 32 + kLoadThreads;   // 480
+constexpr int kLoadThreads = 96;        // a warp of 16-byte gathers moves ~12 B per cycle
+constexpr int kThreads = kSoftmaxThreads + kEpiThreads + 32 + kLoadThreads;   // 512
 constexpr int NK = 2;                   // K pipeline stages
 constexpr int NV = 2;                   // V pipeline stages
 constexpr int kTextChunk = 64;          // kept blocks per work item of a text query row
@@ -219,14 +219,16 @@ __device__ inline float ex2(float x) {
     return y;
 }
 
-// Loader thread lt owns 16-byte chunk (lt % CH) of TPT consecutive rows of a tile: rows
-// (lt / CH) * TPT + k. Its tokens come from the block-slot table in TPT/4 int4 loads, so
+// Loader thread lt owns 16-byte chunk (lt % CH) of up to TPT consecutive rows of a tile: rows
+// (lt / CH) * TPT + k below ROWS (G = kLoadThreads / CH row groups; the last one may be
+// shorter). Its tokens come from the block-slot table in independent loads issued together, so
 // one tile's tokens are a single round trip; K and V of a block share them.
 template <int D, int ROWS>
 struct RowToks {
     static constexpr int CH = D / 8;                      // 16-byte chunks per row
-    static constexpr int TPT = ROWS * CH / kLoadThreads;  // rows per loader thread
-    static_assert(TPT % 4 == 0, "whole int4 loads");
+    static constexpr int G = kLoadThreads / CH;           // row groups
+    static constexpr int TPT = (ROWS + G - 1) / G;        // rows per loader thread (at most)
+    static_assert(kLoadThreads % CH == 0, "whole rows per loader pass");
     int t[TPT];
 };
 
@@ -240,13 +242,10 @@ __device__ inline RowToks<D, ROWS> load_tokens(const int* table, int B, int N, i
     RT rt;
     const int r0 = (lt / RT::CH) * RT::TPT;
 #pragma unroll
-    for (int v = 0; v < RT::TPT / 4; ++v) {
-        int4 q = make_int4(0, 0, 0, 0);
-        if (r0 + 4 * v < B) q = __ldg(reinterpret_cast<const int4*>(table + block * B + r0 + 4 * v));
-        rt.t[4 * v + 0] = min(max(q.x, 0), N - 1);
-        rt.t[4 * v + 1] = min(max(q.y, 0), N - 1);
-        rt.t[4 * v + 2] = min(max(q.z, 0), N - 1);
-        rt.t[4 * v + 3] = min(max(q.w, 0), N - 1);
+    for (int k = 0; k < RT::TPT; ++k) {
+        const int r = r0 + k;
+        const int q = (r < ROWS && r < B) ? __ldg(table + block * B + r) : 0;
+        rt.t[k] = min(max(q, 0), N - 1);
     }
     return rt;
 }
@@ -259,7 +258,8 @@ __device__ inline void gather_tile(const RowToks<D, ROWS>& rt, const bsa_bf16* h
     const int r0 = (lt / RT::CH) * RT::TPT;
 #pragma unroll
     for (int k = 0; k < RT::TPT; ++k)
-        cp_async_16(tile_smem + sw128_offset(ROWS, r0 + k, c), head_base + (size_t)rt.t[k] * D + c * 8);
+        if (r0 + k < ROWS)
+            cp_async_16(tile_smem + sw128_offset(ROWS, r0 + k, c), head_base + (size_t)rt.t[k] * D + c * 8);
 }
 
 #ifdef BSA_TEST_HOOKS
