@@ -152,8 +152,7 @@ def test_scores_tensor_core_path_match_oracle(name):
 
 
 # PARK's one-pass kernel with the key blocks of a head split over a cluster of CTAs: nb above
-# one CTA's share (176 key blocks for d = 128, 256 for d = 64), a partial last chunk, text
-# blocks. The two-pass kernel runs on the same inputs, and a masked head stays untouched.
+# one CTA's share (160 key blocks), a partial last chunk, text blocks. The two-pass kernel runs on the same inputs, and a masked head stays untouched.
 PARK_CLUSTER = {
     "c3_d128_b64_text": dict(heads=2, d=128, T=8, H=48, W=60, text=100, B=64, p=0.9),   # nb 362: 3 x 128
     "c2_d64_b64": dict(heads=2, d=64, T=9, H=32, W=60, text=0, B=64, p=0.9),             # nb 270: 2 x 144
@@ -795,6 +794,35 @@ def test_drift_pass_writes_block_means(name, force):
         bnd = PT.score_bound(Qh, Kh, c.layout, "meanpool", ref)
         _check_scores(S1[h].cpu().numpy(), ref, bnd, ("block means", name, h))
         _check_scores(S2[h].cpu().numpy(), ref, bnd, ("pooled in the call", name, h))
+
+
+def test_drift_block_means_through_key_table():
+    """With a key table the drift pass pools K over the query-aware key blocks (and Q over the
+    tile blocks); the scores taken from those means match the oracle on the same key layout."""
+    bsa = _bsa()
+    c = Case(**SMALL["text_d128_b128"])
+    table, _ = _gpu_cluster(c, 2)
+    means = torch.full((2, c.heads, c.nb, c.d), float("nan"), dtype=torch.float32, device="cuda")
+    prob = bsa.problem(c.heads, c.d, 6, 20, 24, 256, c.B, key_table=table, block_means=means)
+    plan = bsa.bsa_plan(prob)
+    Qr, Kr = PT.to_dev_bf16(c.Qb), PT.to_dev_bf16(c.Kb)
+    drift = torch.zeros(c.heads, dtype=torch.float32, device="cuda")
+    refresh = torch.zeros(c.heads, dtype=torch.int32, device="cuda")
+    bsa.bsa_drift_check(prob, c.Q, c.K, Qr, Kr, 0.05, 1, drift, refresh, c.ws(plan.drift_workspace_bytes))
+    S = torch.empty(c.heads, c.nb, c.nb, dtype=torch.float32, device="cuda")
+    bsa.bsa_score_blocks(prob, c.Q, c.K, None, S, c.ws(plan.score_workspace_bytes))
+    _status_ok()
+    m, tab, S = means.cpu().numpy(), table.cpu().numpy(), S.cpu().numpy()
+    for h in range(c.heads):
+        Qh, Kh = O.bf16_to_f64(c.Qb[h]), O.bf16_to_f64(c.Kb[h])
+        KL = O.key_layout(c.layout, tab[h])
+        for X, L, got in ((Qh, c.layout, m[0, h]), (Kh, KL, m[1, h])):
+            exact = O.pool_blocks(X, L)
+            tol = 64 * PT.U32 * O.pool_blocks(np.abs(X), L)
+            assert np.all(np.abs(got - exact) <= tol), (h, float(np.abs(got - exact).max()))
+        ref = O._softmax_rows(O.pool_blocks(Qh, c.layout) @ O.pool_blocks(Kh, KL).T / math.sqrt(c.d))
+        bnd = PT.score_bound(Qh, Kh, c.layout, "meanpool", ref, klayout=KL)
+        _check_scores(S[h], ref, bnd, ("block means, key table", h))
 
 
 def _grid(name):
