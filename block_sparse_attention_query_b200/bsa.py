@@ -50,6 +50,7 @@ class PlanInfo(ctypes.Structure):
         ("attention_workspace_bytes", ctypes.c_size_t),
         ("mass_workspace_bytes", ctypes.c_size_t),
         ("cluster_workspace_bytes", ctypes.c_size_t),
+        ("park_cluster", ctypes.c_int), ("park_cols", ctypes.c_int),
     ]
 
 

@@ -421,6 +421,11 @@ int bsa_plan(const bsa_problem* prob, bsa_plan_info* out) {
     info.attention_workspace_bytes = attention_ws_bytes(g);
     info.mass_workspace_bytes = mass_ws_bytes(g);
     info.cluster_workspace_bytes = cluster_ws_bytes(g);
+    int pc = 0, pw = 0;
+    if (park_cluster_shape(g, &pc, &pw)) {
+        info.park_cluster = pc;
+        info.park_cols = pw;
+    }
     *out = info;
     return BSA_OK;
 }
@@ -785,7 +790,7 @@ const char* bsa_error_string(int status) {
     }
 }
 
-const char* bsa_version(void) { return "bsa 0.2.0 sm_100a"; }
+const char* bsa_version(void) { return "bsa 0.3.0 sm_100a"; }
 
 int bsa_set_park_kernel(int which) {
     if (which != BSA_PARK_AUTO && which != BSA_PARK_TWO_PASS) return BSA_ERR_ARG;

@@ -109,6 +109,9 @@ typedef struct bsa_plan_info {
     size_t attention_workspace_bytes;  /* bsa_sparse_attention */
     size_t mass_workspace_bytes;       /* bsa_captured_mass */
     size_t cluster_workspace_bytes;    /* bsa_cluster_keys */
+    int park_cluster;   /* PARK scorer under BSA_PARK_AUTO: CTAs per thread-block cluster of the
+                           one-pass kernel (1..8), or 0 when nb needs the two-pass kernel */
+    int park_cols;      /* key blocks each CTA of that cluster holds (0 with park_cluster 0) */
 } bsa_plan_info;
 
 /* Validate `prob` and fill `out`. Host only; launches nothing.
@@ -287,7 +290,7 @@ const char* bsa_error_string(int status);
 #define BSA_PARK_TWO_PASS 1
 int bsa_set_park_kernel(int which);
 
-/* Library version, e.g. "bsa 0.2.0 sm_100a". */
+/* Library version, e.g. "bsa 0.3.0 sm_100a". */
 const char* bsa_version(void);
 
 /* Number of kernels this library has launched in this process so far (all devices, all

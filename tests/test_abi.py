@@ -32,6 +32,20 @@ def test_exports_every_declared_symbol():
         assert n in bsa.EXPORTS, n
 
 
+def test_plan_reports_the_park_cluster_shape():
+    # key blocks split over C CTAs of W (a multiple of 16, at most 160): (C - 1) * W < nb <= C * W
+    for (T, H, W, text, heads), (C, cols) in {(21, 30, 52, 0, 12): (2, 128),      # nb 256
+                                             (21, 45, 80, 0, 40): (4, 160),      # nb 591
+                                             (33, 45, 80, 256, 24): (6, 160),    # nb 931
+                                             (2, 8, 8, 0, 1): (1, 16)}.items():  # nb 1
+        plan = bsa.bsa_plan(bsa.problem(heads, 128, T, H, W, text, 128, score_mode=bsa.BSA_SCORE_PARK))
+        assert (plan.park_cluster, plan.park_cols) == (C, cols), (plan.nb, plan.park_cluster, plan.park_cols)
+        assert (C - 1) * cols < plan.nb <= C * cols and cols % 16 == 0 and cols <= 160
+    # above 8 x 160 key blocks the two-pass kernel runs
+    plan = bsa.bsa_plan(bsa.problem(1, 64, 41, 64, 80, 0, 128, score_mode=bsa.BSA_SCORE_PARK))
+    assert plan.nb > 1280 and plan.park_cluster == 0 and plan.park_cols == 0
+
+
 def test_park_kernel_setting_is_checked_on_the_host():
     # a process-wide host setting: no CUDA call, so it runs without a GPU
     assert bsa.bsa_set_park_kernel(bsa.PARK_TWO_PASS) == 0
