@@ -124,7 +124,7 @@ int park_nbp(const Geom& g) {
 size_t ksplit_bytes(const Geom& g) { return align256((size_t)g.heads * 3 * park_nbp(g) * g.d * 2); }
 int mp_nbq(const Geom& g) { return (g.nb + mp::BQ - 1) / mp::BQ * mp::BQ; }
 size_t qsplit_bytes(const Geom& g) { return align256((size_t)g.heads * 3 * mp_nbq(g) * g.d * 2); }
-size_t rowoff_bytes(const Geom& g) { return align256((size_t)g.heads * g.nb * sizeof(float)); }
+size_t rowoff_bytes(const Geom& g) { return align256((size_t)g.heads * g.nb * 2 * sizeof(float)); }
 size_t score_ws_bytes(const Geom& g, int mode) {
     return pooled_bytes(g) + perm_bytes(g) + ksplit_bytes(g) +
            (mode == BSA_SCORE_MEANPOOL ? qsplit_bytes(g) + rowoff_bytes(g) : 0);
@@ -243,12 +243,17 @@ int launch_meanpool(const Geom& g, const float* qbar, const float* kbar, const i
     P.rowoff = rowoff;
     P.nbq = nbq;
     P.nbp = nbp;
-    P.n_items = g.heads * (nbq / mp::BQ);
+    // too few (head, query tile) items to fill the SMs twice: each item's key tiles in two
+    // halves, the halves' log-sum-exps combined by the normalisation pass
+    const int base_items = g.heads * (nbq / mp::BQ), ntiles = nbp / mp::NT;
+    P.nsplit = (base_items < 2 * sms && ntiles >= 2) ? 2 : 1;
+    P.tps = (ntiles + P.nsplit - 1) / P.nsplit;
+    P.n_items = base_items * P.nsplit;
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     const int grid = P.n_items < sms ? P.n_items : sms;
     mp::meanpool_tc_kernel<D><<<grid, mp::kThreads, C::SMEM, st>>>(P);
     if (launch_status() != BSA_OK) return BSA_ERR_CUDA;
-    mp::normalize_rows_kernel<<<g.heads * g.nb, 128, 0, st>>>(g, head_mask, rowoff, scores);
+    mp::normalize_rows_kernel<<<g.heads * g.nb, 128, 0, st>>>(g, head_mask, rowoff, P.nsplit, scores);
     return launch_status();
 }
 

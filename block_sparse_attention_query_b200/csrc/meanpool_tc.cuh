@@ -11,12 +11,14 @@
 // accumulate in fp32 TMEM; the dropped terms are of order 2^-24 of the logit, the size of a
 // float32 rounding.
 //
-// Persistent kernel, one CTA per SM, work item = (head, tile of 128 pooled query rows). Key
-// blocks come in tiles of 64 (one MMA N), one pass: per tile, each query row's scaled logits
-// (log2 units) go to the output row through a padded staging tile (each store instruction
-// writes 32 consecutive entries of one row) while the row keeps an online max m and sum l of
-// 2^logit; after the last tile the row's offset -(m + log2 l) goes to rowoff, and
-// normalize_rows_kernel rewrites every row as 2^(logit + offset).
+// Persistent kernel, one CTA per SM, work item = (head, tile of 128 pooled query rows, share of
+// the key tiles: all of them, or one of two halves when there are too few items to fill the
+// SMs twice). Key blocks come in tiles of 64 (one MMA N), one pass: per tile, each query row's
+// scaled logits (log2 units) go to the output row through a padded staging tile (each store
+// instruction writes 32 consecutive entries of one row) while the row keeps an online max m and
+// sum l of 2^logit; after the item's last tile the row's log-sum-exp m + log2 l over its share
+// goes to rowoff, and normalize_rows_kernel combines the shares and rewrites every row as
+// 2^(logit - lse).
 // Roles (224 threads): warps 0-3 softmax (thread r = pooled query row r = TMEM lane r), warp 4
 // MMA issuer + TMEM allocation, warps 5-6 loaders (contiguous split rows, 16-byte cp.async).
 // Every wait is bounded.
@@ -69,10 +71,12 @@ struct Params {
     const bsa_bf16* ksplit;   // [heads][3][nbp][D] bf16: hi, mid, lo of the pooled keys
     const int* head_mask;
     float* scores;
-    float* rowoff;            // [heads][nb] -(m + log2 l) of each row
+    float* rowoff;            // [heads][nb][nsplit] log-sum-exp (log2 units) of each row's share
+    int nsplit;               // shares of the key tiles per (head, query tile): 1 or 2
+    int tps;                  // key tiles per share
     int nbq;                  // nb rounded up to a multiple of BQ
     int nbp;                  // nb rounded up to a multiple of NT
-    int n_items;              // heads * nbq / BQ
+    int n_items;              // heads * nbq / BQ * nsplit
     float scale_log2;         // log2(e) / sqrt(d)
 };
 
@@ -128,8 +132,16 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
     const uint32_t sK = smem_u32(sm + C::OFF_K);
 
     auto skip_item = [&](int item) -> bool {
-        const int h = item / qtiles;
+        const int h = item / (qtiles * P.nsplit);
         return P.head_mask != nullptr && P.head_mask[h] == 0;
+    };
+    // item -> head, query tile, key tiles [t0, t1)
+    auto decode = [&](int item, int& h, int& qt, int& t0, int& t1) {
+        const int sp = item % P.nsplit, hq = item / P.nsplit;
+        h = hq / qtiles;
+        qt = hq - h * qtiles;
+        t0 = sp * P.tps;
+        t1 = min(ntiles, t0 + P.tps);
     };
 
     if (warp >= kLoadWarp0) {
@@ -141,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
         int gt = 0, k = 0;
         for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
             if (skip_item(item)) continue;
-            const int h = item / qtiles, qt = item - h * qtiles;
+            int h, qt, t0, t1;
+            decode(item, h, qt, t0, t1);
             if (k >= 1) ok = mbar_wait(q_empty, (k - 1) & 1, epoch);
             if (!ok) break;
             const bsa_bf16* qh = P.qsplit + (size_t)h * 3 * P.nbq * D;
@@ -153,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             }
             cp_async_arrive_noinc(q_full);
             const bsa_bf16* kh = P.ksplit + (size_t)h * 3 * P.nbp * D;
-            for (int t = 0; t < ntiles && ok; ++t, ++gt) {
+            for (int t = t0; t < t1 && ok; ++t, ++gt) {
                 const int s = gt % NS;
                 if (gt >= NS) ok = mbar_wait(&k_empty[s], ((gt / NS) - 1) & 1, epoch);
                 if (!ok) break;
@@ -176,8 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
             int gt = 0, k = 0;
             for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
                 if (skip_item(item)) continue;
+                int h, qt, t0, t1;
+                decode(item, h, qt, t0, t1);
                 ok = mbar_wait(q_full, k & 1, epoch);
-                for (int t = 0; t < ntiles && ok; ++t, ++gt) {
+                for (int t = t0; t < t1 && ok; ++t, ++gt) {
                     const int s = gt % NS, lb = gt & 1;
                     ok = mbar_wait(&k_full[s], (gt / NS) & 1, epoch);
                     if (ok && gt >= 2) ok = mbar_wait(&l_free[lb], ((gt >> 1) - 1) & 1, epoch);
@@ -196,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
                     }
                     tc_commit(&l_full[lb]);
                     tc_commit(&k_empty[s]);
-                    if (t == ntiles - 1) tc_commit(q_empty);
+                    if (t == t1 - 1) tc_commit(q_empty);
                 }
                 ++k;
             }
@@ -212,12 +227,14 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
         int gt = 0;
         for (int item = blockIdx.x; item < P.n_items && ok; item += gridDim.x) {
             if (skip_item(item)) continue;
-            const int h = item / qtiles, qt = item - h * qtiles;
+            int h, qt, t0, t1;
+            decode(item, h, qt, t0, t1);
+            const int sp = item % P.nsplit;
             float m = -INFINITY, l = 0.f;
             const int lane = r & 31;
             float* stg = reinterpret_cast<float*>(sm + C::OFF_STG) + warp * 32 * 33;
             const int row0 = qt * BQ + warp * 32;           // the warp's first query block
-            for (int t = 0; t < ntiles && ok; ++t, ++gt) {
+            for (int t = t0; t < t1 && ok; ++t, ++gt) {
                 const int lb = gt & 1;
                 ok = __all_sync(0xffffffffu, mbar_wait(&l_full[lb], (gt >> 1) & 1, epoch));
                 if (!ok) break;
@@ -260,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
                 }
             }
             if (!ok) break;
-            if (row0 + lane < nb) P.rowoff[(size_t)h * nb + row0 + lane] = -(m + __log2f(l));
+            if (row0 + lane < nb) P.rowoff[((size_t)h * nb + row0 + lane) * P.nsplit + sp] = m + __log2f(l);
         }
     }
 
@@ -273,14 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1) meanpool_tc_kernel(Params P) {
 }
 
 // grid (heads * nb), 128 threads: row (h, i) of the scores, logits (log2 units) ->
-// probabilities 2^(logit + rowoff). Skips heads that were not scored.
+// probabilities 2^(logit - lse), lse combining the row's nsplit shares (each share holds at
+// least one real key block). Skips heads that were not scored.
 __global__ void __launch_bounds__(128) normalize_rows_kernel(Geom g, const int* __restrict__ head_mask,
-                                                             const float* __restrict__ rowoff,
+                                                             const float* __restrict__ rowoff, int nsplit,
                                                              float* __restrict__ scores) {
     const int row = blockIdx.x;
     const int h = row / g.nb;
     if (head_mask != nullptr && head_mask[h] == 0) return;
-    const float off = rowoff[row];
+    float lse = rowoff[(size_t)row * nsplit];
+    if (nsplit == 2) {
+        const float b = rowoff[(size_t)row * nsplit + 1];
+        const float mx = fmaxf(lse, b);
+        lse = mx + __log2f(park::ex2(lse - mx) + park::ex2(b - mx));
+    }
+    const float off = -lse;
     float* p = scores + (size_t)row * g.nb;
     for (int j = threadIdx.x; j < g.nb; j += 128) p[j] = park::ex2(p[j] + off);
 }

@@ -132,7 +132,7 @@ int bsa_block_layout(const bsa_problem* prob, int* perm_host);
  *              key blocks j (including text blocks); logits are scaled by 1/sqrt(d).
  *   ws         workspace of at least plan.score_workspace_bytes: pooled block means, the
  *              block-slot table, the bf16 three-way splits of the pooled keys (and, for the
- *              mean-pooled mode, of the pooled queries and one offset per score row). Its
+ *              mean-pooled mode, of the pooled queries and two log-sum-exps per score row). Its
  *              size depends on the mode, so plan with the mode that will run.
  * Mode is prob->score_mode. Mean-pooled scores are float32-grade: float32 dot products on
  * CUDA cores for problems too small to fill the GPU, otherwise tensor-core products of the

@@ -30,7 +30,7 @@ def test_score_workspace_covers_every_buffer(name):
     perm = nb * w.block * 4                      # block-slot table
     ksplit = h * 3 * _up(nb, 64) * d * 2         # hi/mid/lo bf16 of k-bar, key tiles of 64
     qsplit = h * 3 * _up(nb, 128) * d * 2        # hi/mid/lo bf16 of q-bar, query tiles of 128
-    rowoff = h * nb * 4                          # one softmax offset per score row
+    rowoff = h * nb * 2 * 4                      # two log-sum-exps per score row (key-tile halves)
     assert pk.score_workspace_bytes >= pooled + perm + ksplit
     assert mp.score_workspace_bytes >= pooled + perm + ksplit + qsplit + rowoff
     assert mp.score_workspace_bytes > pk.score_workspace_bytes
